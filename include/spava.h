@@ -1,0 +1,165 @@
+/*
+ * spava.h -- C ABI of libspava: B200 (sm_100a) kernels for the per-host
+ * approximate attention of APB-V / Spava long-video prefill, with every ZigZag
+ * virtual host on one GPU.
+ *
+ * Method source: "Riepilogo Tecnico: APB-V" (gist.science/it/paper/2601.21444),
+ * section "Metodologia: APB-V" -- 1. "Design del Framework" (context split into
+ * anchor block, query block and context blocks; ZigZag pairing of virtual hosts
+ * h and 2H-1-h; passing blocks of the most essential KV found by query-to-context
+ * attention scores; attention over anchor, local context, aggregated passing
+ * blocks and query) and 2. "Ottimizzazioni a Livello di Sistema" ("Forward Fuso
+ * di Contesto e Query": query partial results merged through log-sum-exp;
+ * "Bilanciamento del Carico dell'Attenzione Approssimata").  Also "Spava:
+ * Accelerating Long-Video Understanding via Sequence-Parallelism-aware
+ * Approximate Attention", abstract.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are DEVICE pointers unless the name says host, contiguous,
+ *     token-major: Q [N, Hq, d], K and V [N, Hkv, d], O [N, Hq, d], all bf16
+ *     (passed as void*), and 16-byte aligned.  lse is float32 [Hq, N], natural
+ *     log.  scores are float32 [Hkv, C], C = N - a - q, context token t at
+ *     column t - a.  idx is int32 [2H-1, Hkv, l]: absolute token positions,
+ *     ascending, padded with -1.  Packed passing K/V are bf16 [Hkv, L, d] with
+ *     L = a + sum_u min(l, n_u): the anchor rows first, then P_0, P_1, ...
+ *   - The caller owns every buffer.  The library allocates no device or host
+ *     memory, frees nothing and never synchronises the stream (except
+ *     spava_device_status, which says so).
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).
+ *   - Arguments are checked before any launch; on error nothing is launched
+ *     and the status says why.  SPAVA_ERR_CUDA means a CUDA runtime call
+ *     failed; spava_last_cuda_error() returns its code (per thread).
+ *   - Kernels never trap.  A wait inside a kernel that exceeds its bound sets a
+ *     flag in the workspace status word and the kernel returns early; read it
+ *     with spava_device_status().
+ *   - Thread-safe: no mutable global state besides per-thread error codes and
+ *     the once-per-process kernel attribute set-up.
+ */
+#ifndef SPAVA_H_
+#define SPAVA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPAVA_OK = 0,
+    SPAVA_ERR_INVALID_ARG = 1, /* a size, offset or pointer is invalid */
+    SPAVA_ERR_UNSUPPORTED = 2, /* valid, but outside what this build runs (d, H) */
+    SPAVA_ERR_MISALIGNED = 3,  /* a device pointer is not 16-byte aligned */
+    SPAVA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
+    SPAVA_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+    SPAVA_ERR_TIMEOUT = 6      /* a kernel-side bounded wait gave up */
+} spava_status;
+
+/* One prefill attention layer.  Sequence split of "Suddivisione del Contesto e
+ * Disposizione ZigZag": [anchor a | 2H context chunks | query block q]. */
+typedef struct {
+    int32_t H;            /* physical hosts = virtual-host pairs; 2H chunks; 1..32 */
+    int32_t n_q_heads;    /* Hq */
+    int32_t n_kv_heads;   /* Hkv; Hq % Hkv == 0, q-head h uses KV head h / (Hq/Hkv) */
+    int32_t head_dim;     /* d: 64 or 128 */
+    int64_t n_tokens;     /* N < 2^31 */
+    int64_t anchor_len;   /* a >= 0 */
+    int64_t query_len;    /* q >= 1 */
+    const int64_t *chunk_offsets; /* HOST array [2H+1]: off[0]=a, off[2H]=N-q,
+                                     strictly increasing; chunk v = [off[v], off[v+1]) */
+    int32_t top_l;        /* l >= 0: passing-block size per KV head per chunk */
+    float scale;          /* softmax scale; <= 0 selects 1/sqrt(d) */
+    int32_t local_pair_full; /* 1: the later virtual host of a ZigZag pair sees its
+                                partner chunk in full and takes no passing block from
+                                it; 0: every virtual host takes the passing blocks of
+                                all earlier chunks and no full partner chunk */
+} spava_config;
+
+/* Workspace bytes that any entry point below needs for this config (the
+ * largest of them: spava_prefill_attention).  Pass the same buffer to every
+ * call; it must be 256-byte aligned. */
+spava_status spava_workspace_size(const spava_config *cfg, size_t *bytes);
+
+/* L = a + sum_u min(l, n_u): rows of the packed passing K/V per KV head. */
+spava_status spava_packed_len(const spava_config *cfg, int64_t *rows);
+
+/* Query-to-context scores ("Blocchi di Passaggio"): for every chunk u < 2H-1,
+ * KV head g and key j of chunk u,
+ *   scores[g, j-a] = sum_{h in group g} sum_{i in query block}
+ *                    softmax_{j' in chunk u}(scale * q_{h,i} . k_{g,j'}) at j'=j.
+ * The softmax runs over chunk u only; no causal mask.  The last chunk has no
+ * successor and its columns are left untouched.  Two passes over K: row
+ * statistics, then probability column sums.  Reads q, k; writes scores. */
+spava_status spava_score(const spava_config *cfg, const void *q, const void *k, float *scores,
+                         void *ws, size_t ws_bytes, void *stream);
+
+/* Passing-block selection ("Blocchi di Passaggio": the most essential KV): for
+ * every chunk u < 2H-1 and KV head g, the min(l, n_u) largest scores of chunk u
+ * (ties: the lower token index wins), written as ascending absolute positions
+ * into idx[u, g, :], the remaining slots set to -1.  Exact: no approximation
+ * in the selection. */
+spava_status spava_topk_select(const spava_config *cfg, const float *scores, int32_t *idx,
+                               void *stream);
+
+/* Passing-block aggregation ("aggregate in blocchi di passaggio"): pk[g, r] =
+ * k[r, g] for r < a (anchor), then for each chunk u the rows k[idx[u,g,s], g],
+ * s < min(l, n_u), in that order; pv likewise from v.  On one GPU this gather
+ * replaces the cross-host transfer of the passing blocks. */
+spava_status spava_pack_passing(const spava_config *cfg, const void *k, const void *v,
+                                const int32_t *idx, void *pk, void *pv, void *stream);
+
+/* Approximate attention ("Computazione") with online softmax:
+ *   anchor row t < a:        keys [0, t]
+ *   context row t, chunk v:  anchor + passing blocks of the earlier chunks
+ *                            (local_pair_full=1: those on another physical host)
+ *                            + partner chunk 2H-1-v in full (v >= H,
+ *                            local_pair_full=1) + own chunk up to t
+ *   query row t >= N-q:      keys [0, t], computed as one partial per segment
+ *                            (anchor, each chunk, query block) merged by
+ *                            log-sum-exp ("Forward Fuso di Contesto e Query").
+ * Writes o [N, Hq, d] bf16 and, if lse != NULL, lse [Hq, N] float32. */
+spava_status spava_attn(const spava_config *cfg, const void *q, const void *k, const void *v,
+                        const void *pk, const void *pv, void *o, float *lse, void *ws,
+                        size_t ws_bytes, void *stream);
+
+/* The whole layer: spava_score -> spava_topk_select -> spava_pack_passing ->
+ * spava_attn, with scores, idx and the packed K/V kept in the workspace.  If
+ * idx_out != NULL the passing-block indices are also written there. */
+spava_status spava_prefill_attention(const spava_config *cfg, const void *q, const void *k,
+                                     const void *v, void *o, float *lse, int32_t *idx_out,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/* spava_prefill_attention from HOST buffers: copies q_host, k_host, v_host
+ * into the caller's device buffers q, k, v, runs the layer, and copies o (and
+ * lse if both lse and lse_host are non-NULL) back to o_host / lse_host, all
+ * ordered on `stream`.  Host buffers should be page-locked for the copies to be
+ * asynchronous; the call does not wait for them. */
+spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q_host,
+                                          const void *k_host, const void *v_host, void *o_host,
+                                          float *lse_host, void *q, void *k, void *v, void *o,
+                                          float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, reads the workspace status word (bit 0: a bounded wait
+ * in a kernel gave up), writes it to *flags and clears it.  Returns
+ * SPAVA_ERR_TIMEOUT if bit 0 was set, SPAVA_OK otherwise. */
+spava_status spava_device_status(void *ws, size_t ws_bytes, void *stream, int32_t *flags);
+
+/* Exact number of (row, key) pairs per query head that spava_attn attends,
+ * by row class: pairs[0] anchor rows, pairs[1] context rows, pairs[2] query
+ * rows.  Algorithmic FLOPs of spava_attn = 4 * d * Hq * (sum of the three).
+ * per_host (may be NULL) receives H entries: the context pairs of each
+ * physical host, i.e. of its two virtual hosts p and 2H-1-p (ZigZag balance,
+ * "Bilanciamento del Carico dell'Attenzione Approssimata").  Host only. */
+spava_status spava_attended_pairs(const spava_config *cfg, int64_t pairs[3], int64_t *per_host);
+
+const char *spava_status_string(spava_status s);
+
+/* The CUDA error code of this thread's last SPAVA_ERR_CUDA (0 if none). */
+int32_t spava_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPAVA_H_ */

@@ -1,0 +1,188 @@
+"""PyTorch-facing wrappers of the libspava C ABI (same names as include/spava.h).
+
+Argument marshalling only: shapes and dtypes are checked, pointers and the
+current CUDA stream are handed to the library, and every step of the
+computation runs in the library's kernels.  PyTorch provides device memory and
+streams.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+from . import native
+from .native import SpavaConfig
+
+
+@dataclass
+class Layout:
+    """One prefill attention layer: [anchor a | 2H chunks | query q]."""
+    H: int
+    Hq: int
+    Hkv: int
+    d: int
+    N: int
+    a: int
+    q: int
+    offsets: np.ndarray
+    l: int
+    scale: float = 0.0
+    local_pair_full: int = 1
+    _keep: list = field(default_factory=list, repr=False)
+
+    @classmethod
+    def from_workload(cls, w, offsets=None) -> "Layout":
+        from .synth import chunk_offsets
+        off = chunk_offsets(w) if offsets is None else offsets
+        return cls(w.H, w.Hq, w.Hkv, w.d, w.N, w.a, w.q, np.asarray(off, dtype=np.int64), w.l,
+                   0.0, w.local_pair_full)
+
+    def c(self) -> SpavaConfig:
+        off = np.ascontiguousarray(self.offsets, dtype=np.int64)
+        self._keep = [off]
+        return SpavaConfig(self.H, self.Hq, self.Hkv, self.d, self.N, self.a, self.q,
+                           off.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), self.l,
+                           float(self.scale), int(self.local_pair_full))
+
+    @property
+    def n_chunks(self) -> int:
+        return 2 * self.H
+
+    @property
+    def context(self) -> int:
+        return self.N - self.a - self.q
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(t: torch.Tensor, shape, dtype, name):
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: expected contiguous {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+
+
+def workspace_size(lay: Layout) -> int:
+    n = ctypes.c_size_t()
+    cfg = lay.c()
+    native.call("spava_workspace_size", ctypes.byref(cfg), ctypes.byref(n))
+    return n.value
+
+
+def packed_len(lay: Layout) -> int:
+    n = ctypes.c_int64()
+    cfg = lay.c()
+    native.call("spava_packed_len", ctypes.byref(cfg), ctypes.byref(n))
+    return n.value
+
+
+def attended_pairs(lay: Layout):
+    """(anchor, context, query) attended (row, key) pairs per head, and the
+    context pairs per physical host."""
+    pairs = (ctypes.c_int64 * 3)()
+    per_host = (ctypes.c_int64 * lay.H)()
+    cfg = lay.c()
+    native.call("spava_attended_pairs", ctypes.byref(cfg), pairs, per_host)
+    return tuple(pairs), list(per_host)
+
+
+def new_workspace(lay: Layout, device) -> torch.Tensor:
+    """A zeroed workspace (the status word must start at zero)."""
+    return torch.zeros(workspace_size(lay), dtype=torch.uint8, device=device)
+
+
+class Spava:
+    """A layer layout plus its workspace on one device."""
+
+    def __init__(self, lay: Layout, device="cuda", workspace: torch.Tensor | None = None):
+        self.lay = lay
+        self.device = torch.device(device)
+        self.cfg = lay.c()
+        self.ws = new_workspace(lay, self.device) if workspace is None else workspace
+        self.L = packed_len(lay)
+
+    # -- shapes
+    def _qkv(self, q, k, v=None):
+        lay = self.lay
+        _check(q, (lay.N, lay.Hq, lay.d), torch.bfloat16, "q")
+        _check(k, (lay.N, lay.Hkv, lay.d), torch.bfloat16, "k")
+        if v is not None:
+            _check(v, (lay.N, lay.Hkv, lay.d), torch.bfloat16, "v")
+
+    def _args(self):
+        return ctypes.byref(self.cfg)
+
+    # -- steps
+    def score(self, q, k, scores=None):
+        self._qkv(q, k)
+        lay = self.lay
+        if scores is None:
+            scores = torch.zeros((lay.Hkv, lay.context), dtype=torch.float32, device=self.device)
+        native.call("spava_score", self._args(), _ptr(q), _ptr(k), _ptr(scores), _ptr(self.ws),
+                    self.ws.numel(), _stream(self.device))
+        return scores
+
+    def topk_select(self, scores, idx=None):
+        lay = self.lay
+        _check(scores, (lay.Hkv, lay.context), torch.float32, "scores")
+        if idx is None:
+            idx = torch.empty((lay.n_chunks - 1, lay.Hkv, lay.l), dtype=torch.int32, device=self.device)
+        native.call("spava_topk_select", self._args(), _ptr(scores), _ptr(idx), _stream(self.device))
+        return idx
+
+    def pack_passing(self, k, v, idx, pk=None, pv=None):
+        lay = self.lay
+        shape = (lay.Hkv, self.L, lay.d)
+        pk = torch.empty(shape, dtype=torch.bfloat16, device=self.device) if pk is None else pk
+        pv = torch.empty(shape, dtype=torch.bfloat16, device=self.device) if pv is None else pv
+        native.call("spava_pack_passing", self._args(), _ptr(k), _ptr(v), _ptr(idx), _ptr(pk),
+                    _ptr(pv), _stream(self.device))
+        return pk, pv
+
+    def attn(self, q, k, v, pk, pv, o=None, lse=None, want_lse=True):
+        self._qkv(q, k, v)
+        lay = self.lay
+        o = torch.empty_like(q) if o is None else o
+        if lse is None and want_lse:
+            lse = torch.empty((lay.Hq, lay.N), dtype=torch.float32, device=self.device)
+        native.call("spava_attn", self._args(), _ptr(q), _ptr(k), _ptr(v), _ptr(pk), _ptr(pv),
+                    _ptr(o), _ptr(lse), _ptr(self.ws), self.ws.numel(), _stream(self.device))
+        return o, lse
+
+    def prefill_attention(self, q, k, v, o=None, lse=None, idx_out=None, want_lse=True,
+                          want_idx=False):
+        self._qkv(q, k, v)
+        lay = self.lay
+        o = torch.empty_like(q) if o is None else o
+        if lse is None and want_lse:
+            lse = torch.empty((lay.Hq, lay.N), dtype=torch.float32, device=self.device)
+        if idx_out is None and want_idx:
+            idx_out = torch.empty((lay.n_chunks - 1, lay.Hkv, lay.l), dtype=torch.int32,
+                                  device=self.device)
+        native.call("spava_prefill_attention", self._args(), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                    _ptr(lse), _ptr(idx_out), _ptr(self.ws), self.ws.numel(), _stream(self.device))
+        return o, lse, idx_out
+
+    def prefill_attention_host(self, q_host, k_host, v_host, o_host, lse_host, q, k, v, o, lse):
+        """Host (pinned) buffers in and out; device buffers are the caller's."""
+        native.call("spava_prefill_attention_host", self._args(), _ptr(q_host), _ptr(k_host),
+                    _ptr(v_host), _ptr(o_host), _ptr(lse_host), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                    _ptr(lse), _ptr(self.ws), self.ws.numel(), _stream(self.device))
+
+    def device_status(self) -> int:
+        """Synchronises, returns and clears the kernels' status word (0 = clean)."""
+        flags = ctypes.c_int32()
+        lib = native.load()
+        lib.spava_device_status(_ptr(self.ws), self.ws.numel(), _stream(self.device),
+                                ctypes.byref(flags))
+        return flags.value

@@ -1,0 +1,149 @@
+// plan.cuh -- work items and key segments of the approximate attention, shared
+// by the host planner and the kernels (__host__ __device__, integer only).
+//
+// Sequence split ("Riepilogo Tecnico: APB-V", Metodologia, "Suddivisione del
+// Contesto e Disposizione ZigZag"): [anchor | chunk 0 .. chunk 2H-1 | query].
+// Physical host p holds virtual hosts p and 2H-1-p.
+//
+// Key set of a row ("Meccanismo di Attenzione Approssimata", "Computazione"),
+// expressed as at most four contiguous segments of either the original K/V
+// (src 0, token positions) or the packed passing K/V (src 1, packed rows
+// [anchor | P_0 | P_1 | ...]):
+//   context row t of chunk v:
+//     local_pair_full and v >= H (partner p = 2H-1-v, an earlier chunk):
+//        packed [0, pcum[p])            anchor + P_0..P_{p-1}
+//        packed [pcum[p+1], pcum[v])    P_{p+1}..P_{v-1}
+//        K      [off[p], off[p+1])      the partner chunk in full
+//     otherwise:
+//        packed [0, pcum[v])            anchor + P_0..P_{v-1}
+//     and   K   [off[v], t]             own chunk, causal
+//   anchor row t:  K [0, t]
+//   query rows ("Forward Fuso di Contesto e Query"): one partial per segment
+//     s = 0 anchor [0,a), s = 1+v chunk v, s = 2H+1 query block [N-q, t];
+//     the partials are merged by log-sum-exp afterwards.
+//   score statistics of chunk u: K [off[u], off[u+1]) for the query rows.
+#pragma once
+
+#include <stdint.h>
+
+namespace spava {
+
+constexpr int kMaxChunks = 64;   // 2H <= 64
+constexpr int kMaxGroups = 2 * kMaxChunks + 8 + 2 * kMaxChunks;
+constexpr int kRowTile = 128;    // query rows per work item
+constexpr int kKeyTile = 128;    // keys per pipeline step
+constexpr int kMaxSegs = 4;      // key segments of one work item
+
+enum ItemKind : int32_t { kCtx = 0, kAnchor = 1, kQueryPart = 2, kStats = 3 };
+
+struct Layer {
+    int32_t H, Hq, Hkv, d, G, lpf, l, n_chunks;
+    int32_t N, a, q, C, L;             // tokens, anchor, query, context, packed rows
+    float scale_log2;                  // softmax scale * log2(e)
+    int32_t off[kMaxChunks + 1];       // chunk offsets
+    int32_t pcum[kMaxChunks + 1];      // packed row where P_u starts; pcum[0] = a
+};
+
+// A run of work items of one kind and one chunk/segment; items inside a group
+// are (row tile descending, head ascending) so consecutive CTAs share a KV head.
+struct Group {
+    int32_t kind, sub, n_rt, item_begin;
+};
+
+struct Item {
+    int32_t kind, sub, rt, h;
+};
+
+struct Seg {
+    int32_t src, begin, end, causal;
+};
+
+__host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+__host__ __device__ inline int pair_of(int H, int v) { return v < H ? v : 2 * H - 1 - v; }
+
+__host__ __device__ inline Item decode_item(const Group *groups, int n_groups, int b, int Hq) {
+    int k = 0;
+    while (k + 1 < n_groups && b >= groups[k + 1].item_begin) ++k;
+    const Group &g = groups[k];
+    const int i = b - g.item_begin;
+    Item it;
+    it.kind = g.kind;
+    it.sub = g.sub;
+    it.rt = g.n_rt - 1 - i / Hq;
+    it.h = i % Hq;
+    return it;
+}
+
+// Rows [row0, row_end) of the item.
+__host__ __device__ inline void item_rows(const Layer &L, const Item &it, int &row0, int &row_end) {
+    int lo, hi;
+    if (it.kind == kCtx) {
+        lo = L.off[it.sub];
+        hi = L.off[it.sub + 1];
+    } else if (it.kind == kAnchor) {
+        lo = 0;
+        hi = L.a;
+    } else {
+        lo = L.N - L.q;
+        hi = L.N;
+    }
+    row0 = lo + it.rt * kRowTile;
+    row_end = row0 + kRowTile < hi ? row0 + kRowTile : hi;
+}
+
+__host__ __device__ inline void add_seg(Seg *s, int &n, int src, int b, int e, int causal) {
+    if (e > b) {
+        s[n].src = src;
+        s[n].begin = b;
+        s[n].end = e;
+        s[n].causal = causal;
+        ++n;
+    }
+}
+
+// Segments of the item's key sequence (at most kMaxSegs).  Returns their count.
+__host__ __device__ inline int build_segments(const Layer &L, const Item &it, Seg *s) {
+    int n = 0, row0, row_end;
+    item_rows(L, it, row0, row_end);
+    switch (it.kind) {
+        case kCtx: {
+            const int v = it.sub;
+            if (L.lpf && v >= L.H) {
+                const int p = 2 * L.H - 1 - v;
+                add_seg(s, n, 1, 0, L.pcum[p], 0);
+                add_seg(s, n, 1, L.pcum[p + 1], L.pcum[v], 0);
+                add_seg(s, n, 0, L.off[p], L.off[p + 1], 0);
+            } else {
+                add_seg(s, n, 1, 0, L.pcum[v], 0);
+            }
+            add_seg(s, n, 0, L.off[v], row_end, 1);
+            break;
+        }
+        case kAnchor:
+            add_seg(s, n, 0, 0, row_end, 1);
+            break;
+        case kQueryPart: {
+            const int sg = it.sub;
+            if (sg == 0)
+                add_seg(s, n, 0, 0, L.a, 0);
+            else if (sg <= L.n_chunks)
+                add_seg(s, n, 0, L.off[sg - 1], L.off[sg], 0);
+            else
+                add_seg(s, n, 0, L.N - L.q, row_end, 1);
+            break;
+        }
+        default:  // kStats
+            add_seg(s, n, 0, L.off[it.sub], L.off[it.sub + 1], 0);
+            break;
+    }
+    return n;
+}
+
+__host__ __device__ inline int count_tiles(const Seg *s, int n) {
+    int t = 0;
+    for (int i = 0; i < n; ++i) t += cdiv(s[i].end - s[i].begin, kKeyTile);
+    return t;
+}
+
+}  // namespace spava

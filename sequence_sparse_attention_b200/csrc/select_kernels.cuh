@@ -1,0 +1,204 @@
+// select_kernels.cuh -- passing-block selection, aggregation, and the merge of
+// the query-row partials.
+//
+// "Riepilogo Tecnico: APB-V", Metodologia, "Blocchi di Passaggio": per host,
+// the most essential KV (top-l per KV head by query-to-context score) are
+// aggregated into passing blocks; on one GPU the cross-host transfer of those
+// blocks ("Comunicazione Sovrapposta") becomes the gather in pack_kernel.
+// "Forward Fuso di Contesto e Query": the query rows' per-segment partial
+// results are merged through their log-sum-exp (merge_kernel).
+#pragma once
+
+#include "plan.cuh"
+#include "sm100.cuh"
+
+namespace spava {
+
+// fp32 -> uint32 key whose unsigned order equals the float order.
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix sum over the block (blockDim.x multiple of 32, <= 1024).
+__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int *total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int s = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        if (lane < nw) warp_sums[lane] = s;  // inclusive over warps
+        if (lane == nw - 1) *total = s;
+    }
+    __syncthreads();
+    const int before = (w > 0 ? warp_sums[w - 1] : 0) + x - v;
+    __syncthreads();
+    return before;
+}
+
+// One CTA per (chunk u < 2H-1, KV head g): the min(l, n_u) largest scores of
+// the chunk, ties to the lower token index, written ascending as absolute
+// positions; padding -1.  Radix select on the ordered 32-bit key (4 passes of
+// 8 bits) finds the exact threshold key T and how many keys equal to T are
+// kept; a final pass in index order emits the set, so the output is sorted and
+// the lower-index rule holds for the keys equal to T.
+constexpr int kSelectThreads = 1024;
+
+__global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, const float *scores,
+                                                              int32_t *idx) {
+    __shared__ int hist[256];
+    __shared__ int warp_sums[32];
+    __shared__ int s_digit, s_need, s_total;
+    const int u = blockIdx.x / L.Hkv, g = blockIdx.x % L.Hkv;
+    const int base = L.off[u];
+    const int n = L.off[u + 1] - base;
+    const int l_eff = min(L.l, n);
+    const float *S = scores + static_cast<size_t>(g) * L.C + (base - L.a);
+    int32_t *out = idx + (static_cast<size_t>(u) * L.Hkv + g) * L.l;
+    const int tid = threadIdx.x;
+
+    for (int r = l_eff + tid; r < L.l; r += blockDim.x) out[r] = -1;
+    if (l_eff == 0) return;
+    if (l_eff == n) {
+        for (int r = tid; r < n; r += blockDim.x) out[r] = base + r;
+        return;
+    }
+
+    uint32_t prefix = 0, mask = 0;
+    int need = l_eff;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        if (tid < 256) hist[tid] = 0;
+        __syncthreads();
+        for (int j = tid; j < n; j += blockDim.x) {
+            const uint32_t k = ordered_key(S[j]);
+            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int cum = 0, d = 0;
+            for (int b = 255; b >= 0; --b) {
+                if (cum + hist[b] >= need) {
+                    d = b;
+                    break;
+                }
+                cum += hist[b];
+            }
+            s_digit = d;
+            s_need = need - cum;
+        }
+        __syncthreads();
+        prefix |= static_cast<uint32_t>(s_digit) << shift;
+        mask |= 255u << shift;
+        need = s_need;
+        __syncthreads();
+    }
+    const uint32_t T = prefix;  // key of the l_eff-th largest score
+    const int need_eq = need;   // how many keys equal to T are kept
+
+    const int per = (n + blockDim.x - 1) / blockDim.x;
+    const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
+    int gt = 0, eq = 0;
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t k = ordered_key(S[j]);
+        gt += k > T;
+        eq += k == T;
+    }
+    const int eq_before = block_exclusive_scan(eq, warp_sums, &s_total);
+    const int take_eq = max(0, min(eq, need_eq - eq_before));
+    int pos = block_exclusive_scan(gt + take_eq, warp_sums, &s_total);
+    int taken = 0;
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t k = ordered_key(S[j]);
+        if (k > T || (k == T && taken < take_eq)) {
+            out[pos++] = base + j;
+            taken += (k == T);
+        }
+    }
+}
+
+// Packed passing K/V: row r of KV head g is the anchor row r (r < a) or the
+// s-th kept key of chunk u (r = pcum[u] + s).  One warp per packed row: the
+// first half copies the K row, the second half the V row, 16 bytes per lane.
+template <int D>
+__global__ void __launch_bounds__(256) pack_kernel(const Layer L, const __nv_bfloat16 *K,
+                                                   const __nv_bfloat16 *V, const int32_t *idx,
+                                                   __nv_bfloat16 *PK, __nv_bfloat16 *PV) {
+    constexpr int kChunks = D * 2 / 16;  // 16-byte pieces per row
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long total = static_cast<long long>(L.Hkv) * L.L;
+    if (warp >= total) return;
+    const int g = static_cast<int>(warp / L.L);
+    const int r = static_cast<int>(warp % L.L);
+    int src;
+    if (r < L.a) {
+        src = r;
+    } else {
+        int u = 0;
+        while (u + 1 < L.n_chunks - 1 && r >= L.pcum[u + 1]) ++u;
+        src = idx[(static_cast<size_t>(u) * L.Hkv + g) * L.l + (r - L.pcum[u])];
+    }
+    const int half = lane >> 4, c = lane & 15;
+    if (c >= kChunks) return;
+    __nv_bfloat16 *d = (half ? PV : PK) + (static_cast<size_t>(g) * L.L + r) * D;
+    if (src < 0 || src >= L.N) {  // not a token position: write a zero row, read nothing
+        reinterpret_cast<uint4 *>(d)[c] = make_uint4(0, 0, 0, 0);
+        return;
+    }
+    const __nv_bfloat16 *s = (half ? V : K) + (static_cast<size_t>(src) * L.Hkv + g) * D;
+    reinterpret_cast<uint4 *>(d)[c] = __ldg(reinterpret_cast<const uint4 *>(s) + c);
+}
+
+// Query rows: O = sum_s w_s O_s / sum_s w_s, w_s = 2^(lse2_s - max), over the
+// segments s present (anchor if a > 0, every chunk, the query block itself).
+// One warp per (head, query row); D/4 lanes hold 4 columns each.
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(const Layer L, const float *part_O,
+                                                    const float *part_lse, __nv_bfloat16 *O,
+                                                    float *lse) {
+    const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= L.Hq * L.q) return;
+    const int h = w / L.q, i = w % L.q;
+    const int n_seg = L.n_chunks + 2;
+    const int s_first = L.a > 0 ? 0 : 1;
+    float m = -INFINITY;
+    for (int s = s_first; s < n_seg; ++s)
+        m = fmaxf(m, part_lse[(static_cast<size_t>(s) * L.Hq + h) * L.q + i]);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float wsum = 0.f;
+    for (int s = s_first; s < n_seg; ++s) {
+        const size_t row = (static_cast<size_t>(s) * L.Hq + h) * L.q + i;
+        const float ws = ex2(part_lse[row] - m);
+        wsum += ws;
+        if (lane < D / 4) {
+            const float4 o = __ldg(reinterpret_cast<const float4 *>(part_O + row * D) + lane);
+            acc[0] += ws * o.x;
+            acc[1] += ws * o.y;
+            acc[2] += ws * o.z;
+            acc[3] += ws * o.w;
+        }
+    }
+    const float inv = 1.f / wsum;
+    const int t = L.N - L.q + i;
+    if (lane < D / 4) {
+        uint2 v;
+        v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        reinterpret_cast<uint2 *>(O + (static_cast<size_t>(t) * L.Hq + h) * D)[lane] = v;
+    }
+    if (lane == 0 && lse) lse[static_cast<size_t>(h) * L.N + t] = (m + __log2f(wsum)) * 0.69314718055994531f;
+}
+
+}  // namespace spava

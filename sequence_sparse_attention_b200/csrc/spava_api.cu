@@ -1,0 +1,521 @@
+// spava_api.cu -- the C ABI (include/spava.h): argument checks, the plan of work
+// items, TMA descriptors, workspace layout and kernel launches.  Every step of
+// the computation runs in the kernels; this file only prepares and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/spava.h"
+#include "attn_kernel.cuh"
+#include "plan.cuh"
+#include "score_kernel.cuh"
+#include "select_kernels.cuh"
+
+using namespace spava;
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+spava_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = static_cast<int32_t>(e);
+    return SPAVA_ERR_CUDA;
+}
+
+#define SPAVA_CUDA(...)                                    \
+    do {                                                   \
+        cudaError_t e_ = (__VA_ARGS__);                           \
+        if (e_ != cudaSuccess) return cuda_fail(e_);       \
+    } while (0)
+
+#define SPAVA_TRY(...)                                     \
+    do {                                                   \
+        spava_status s_ = (__VA_ARGS__);                          \
+        if (s_ != SPAVA_OK) return s_;                     \
+    } while (0)
+
+// ---------------------------------------------------------------- config
+spava_status make_layer(const spava_config *c, Layer *L) {
+    if (!c || !L || !c->chunk_offsets) return SPAVA_ERR_INVALID_ARG;
+    if (c->H < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1 || c->head_dim < 1)
+        return SPAVA_ERR_INVALID_ARG;
+    if (c->n_q_heads % c->n_kv_heads) return SPAVA_ERR_INVALID_ARG;
+    if (c->anchor_len < 0 || c->query_len < 1 || c->top_l < 0 || c->n_tokens < 1)
+        return SPAVA_ERR_INVALID_ARG;
+    if (c->local_pair_full != 0 && c->local_pair_full != 1) return SPAVA_ERR_INVALID_ARG;
+    if (c->H > kMaxChunks / 2) return SPAVA_ERR_UNSUPPORTED;
+    if (c->head_dim != 64 && c->head_dim != 128) return SPAVA_ERR_UNSUPPORTED;
+    if (c->n_tokens >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
+    const int nc = 2 * c->H;
+    const int64_t *off = c->chunk_offsets;
+    if (off[0] != c->anchor_len || off[nc] != c->n_tokens - c->query_len) return SPAVA_ERR_INVALID_ARG;
+    for (int v = 0; v < nc; ++v)
+        if (off[v + 1] <= off[v]) return SPAVA_ERR_INVALID_ARG;
+    std::memset(L, 0, sizeof(*L));
+    L->H = c->H;
+    L->Hq = c->n_q_heads;
+    L->Hkv = c->n_kv_heads;
+    L->d = c->head_dim;
+    L->G = c->n_q_heads / c->n_kv_heads;
+    L->lpf = c->local_pair_full;
+    L->l = c->top_l;
+    L->n_chunks = nc;
+    L->N = static_cast<int32_t>(c->n_tokens);
+    L->a = static_cast<int32_t>(c->anchor_len);
+    L->q = static_cast<int32_t>(c->query_len);
+    L->C = L->N - L->a - L->q;
+    for (int v = 0; v <= nc; ++v) L->off[v] = static_cast<int32_t>(off[v]);
+    L->pcum[0] = L->a;
+    for (int u = 0; u < nc - 1; ++u) {
+        const int n_u = L->off[u + 1] - L->off[u];
+        L->pcum[u + 1] = L->pcum[u] + std::min(L->l, n_u);
+    }
+    L->L = L->pcum[nc - 1];
+    const double scale = c->scale > 0.f ? static_cast<double>(c->scale) : 1.0 / std::sqrt(double(c->head_dim));
+    L->scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+    return SPAVA_OK;
+}
+
+// ---------------------------------------------------------------- plan
+int item_tiles(const Layer &L, const Item &it) {
+    Seg s[kMaxSegs];
+    const int n = build_segments(L, it, s);
+    return count_tiles(s, n);
+}
+
+// Groups of the attention launch, most expensive first: the hardware block
+// scheduler hands out CTAs in index order, so a cost-descending order is a
+// longest-processing-time-first schedule over the SMs.  Inside a group, items
+// run row tile descending (cost descending) with the heads of one KV group
+// adjacent (shared K/V tiles in L2).
+int plan_attention(const Layer &L, bool stats, Group *out) {
+    struct G { Group g; int cost; };
+    std::vector<G> gs;
+    auto push = [&](int kind, int sub, int n_rt) {
+        if (n_rt <= 0) return;
+        Item it{kind, sub, n_rt - 1, 0};
+        gs.push_back({Group{kind, sub, n_rt, 0}, item_tiles(L, it)});
+    };
+    const int n_qrt = cdiv(L.q, kRowTile);
+    if (stats) {
+        for (int u = 0; u < L.n_chunks - 1; ++u) push(kStats, u, n_qrt);
+    } else {
+        for (int v = 0; v < L.n_chunks; ++v) push(kCtx, v, cdiv(L.off[v + 1] - L.off[v], kRowTile));
+        if (L.a > 0) push(kAnchor, 0, cdiv(L.a, kRowTile));
+        for (int s = (L.a > 0 ? 0 : 1); s < L.n_chunks + 2; ++s) push(kQueryPart, s, n_qrt);
+    }
+    std::stable_sort(gs.begin(), gs.end(), [](const G &x, const G &y) { return x.cost > y.cost; });
+    int begin = 0, n = 0;
+    for (auto &g : gs) {
+        g.g.item_begin = begin;
+        begin += g.g.n_rt * L.Hq;
+        out[n++] = g.g;
+    }
+    return n;
+}
+
+int64_t plan_items(const Group *g, int n, int Hq) {
+    return n ? static_cast<int64_t>(g[n - 1].item_begin) + static_cast<int64_t>(g[n - 1].n_rt) * Hq : 0;
+}
+
+// ---------------------------------------------------------------- workspace
+struct WsLayout {
+    size_t status, stats, scores, idx, pk, pv, part_o, part_lse, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+WsLayout ws_layout(const Layer &L) {
+    WsLayout w{};
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+    w.status = take(256);
+    w.stats = take(sizeof(float) * size_t(L.n_chunks - 1) * L.Hq * L.q);
+    w.scores = take(sizeof(float) * size_t(L.Hkv) * L.C);
+    w.idx = take(sizeof(int32_t) * size_t(L.n_chunks - 1) * L.Hkv * L.l);
+    w.pk = take(2 * size_t(L.Hkv) * L.L * L.d);
+    w.pv = take(2 * size_t(L.Hkv) * L.L * L.d);
+    w.part_o = take(sizeof(float) * size_t(L.n_chunks + 2) * L.Hq * L.q * L.d);
+    w.part_lse = take(sizeof(float) * size_t(L.n_chunks + 2) * L.Hq * L.q);
+    w.total = o;
+    return w;
+}
+
+spava_status check_ws(const Layer &L, void *ws, size_t ws_bytes) {
+    if (!ws) return SPAVA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return SPAVA_ERR_MISALIGNED;
+    if (ws_bytes < ws_layout(L).total) return SPAVA_ERR_WORKSPACE;
+    return SPAVA_OK;
+}
+
+spava_status check_ptr(const void *p, bool required = true) {
+    if (!p) return required ? SPAVA_ERR_INVALID_ARG : SPAVA_OK;
+    return (reinterpret_cast<uintptr_t>(p) & 15) ? SPAVA_ERR_MISALIGNED : SPAVA_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+spava_status get_encoder(EncodeTiledFn *fn) {
+    std::call_once(g_encode_once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(p);
+        else if (g_encode_err == cudaSuccess)
+            g_encode_err = cudaErrorSymbolNotFound;
+    });
+    if (!g_encode) return cuda_fail(g_encode_err);
+    *fn = g_encode;
+    return SPAVA_OK;
+}
+
+// bf16 3-D map {d0 inner, d1, d2}, 128-byte swizzle, zero fill out of bounds.
+spava_status encode_3d(CUtensorMap *tm, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint32_t b0, uint32_t b1, uint32_t b2) {
+    EncodeTiledFn fn;
+    SPAVA_TRY(get_encoder(&fn));
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = static_cast<int32_t>(r);
+        return SPAVA_ERR_CUDA;
+    }
+    return SPAVA_OK;
+}
+
+// Token-major [N, H, D] tensor, boxes of 64 columns x 1 head x 128 tokens.
+spava_status map_tokens(CUtensorMap *tm, const void *p, const Layer &L, int heads) {
+    return encode_3d(tm, p, L.d, heads, L.N, 64, 1, 128);
+}
+// Packed [Hkv, rows, D] tensor, boxes of 64 columns x 128 rows x 1 head.
+spava_status map_packed(CUtensorMap *tm, const void *p, const Layer &L) {
+    return encode_3d(tm, p, L.d, std::max(L.L, 1), L.Hkv, 64, 128, 1);
+}
+
+template <typename K>
+spava_status set_smem(K kernel, int bytes) {
+    SPAVA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+    return SPAVA_OK;
+}
+
+spava_status launched() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SPAVA_OK : cuda_fail(e);
+}
+
+// ---------------------------------------------------------------- launches
+template <int D, bool STATS>
+spava_status launch_attn(AttnParams &p, cudaStream_t st) {
+    using SM = AttnSmem<D, STATS>;
+    const int64_t items = plan_items(p.groups, p.n_groups, p.L.Hq);
+    if (items == 0) return SPAVA_OK;
+    if (items >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
+    SPAVA_TRY(set_smem(attn_kernel<D, STATS>, SM::kAlloc));
+    attn_kernel<D, STATS><<<static_cast<unsigned>(items), kAttnThreads, SM::kAlloc, st>>>(p);
+    return launched();
+}
+
+spava_status run_stats(const Layer &L, const void *q, const void *k, char *ws, cudaStream_t st) {
+    const WsLayout w = ws_layout(L);
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.L = L;
+    SPAVA_TRY(map_tokens(&p.tmQ, q, L, L.Hq));
+    SPAVA_TRY(map_tokens(&p.tmK, k, L, L.Hkv));
+    p.n_groups = plan_attention(L, true, p.groups);
+    p.stats = reinterpret_cast<float *>(ws + w.stats);
+    p.status = reinterpret_cast<int *>(ws + w.status);
+    return L.d == 128 ? launch_attn<128, true>(p, st) : launch_attn<64, true>(p, st);
+}
+
+spava_status run_scores(const Layer &L, const void *q, const void *k, float *scores, char *ws,
+                        cudaStream_t st) {
+    const WsLayout w = ws_layout(L);
+    ScoreParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.L = L;
+    SPAVA_TRY(map_tokens(&p.tmQ, q, L, L.Hq));
+    SPAVA_TRY(map_tokens(&p.tmK, k, L, L.Hkv));
+    p.stats = reinterpret_cast<const float *>(ws + w.stats);
+    p.scores = scores;
+    p.status = reinterpret_cast<int *>(ws + w.status);
+    int tiles = 0;
+    for (int u = 0; u < L.n_chunks - 1; ++u) {
+        p.tile_begin[u] = tiles;
+        tiles += cdiv(L.off[u + 1] - L.off[u], 128);
+    }
+    p.tile_begin[L.n_chunks - 1] = tiles;
+    const int64_t blocks = static_cast<int64_t>(tiles) * L.Hkv;
+    if (blocks == 0) return SPAVA_OK;
+    if (L.d == 128) {
+        SPAVA_TRY(set_smem(score_kernel<128>, ScoreSmem<128>::kAlloc));
+        score_kernel<128><<<static_cast<unsigned>(blocks), 192, ScoreSmem<128>::kAlloc, st>>>(p);
+    } else {
+        SPAVA_TRY(set_smem(score_kernel<64>, ScoreSmem<64>::kAlloc));
+        score_kernel<64><<<static_cast<unsigned>(blocks), 192, ScoreSmem<64>::kAlloc, st>>>(p);
+    }
+    return launched();
+}
+
+spava_status run_topk(const Layer &L, const float *scores, int32_t *idx, cudaStream_t st) {
+    const int blocks = (L.n_chunks - 1) * L.Hkv;
+    if (blocks == 0 || L.l == 0) return SPAVA_OK;
+    topk_kernel<<<blocks, kSelectThreads, 0, st>>>(L, scores, idx);
+    return launched();
+}
+
+spava_status run_pack(const Layer &L, const void *k, const void *v, const int32_t *idx, void *pk,
+                      void *pv, cudaStream_t st) {
+    const int64_t warps = static_cast<int64_t>(L.Hkv) * L.L;
+    if (warps == 0) return SPAVA_OK;
+    const int64_t blocks = (warps + 7) / 8;
+    auto K = static_cast<const __nv_bfloat16 *>(k);
+    auto V = static_cast<const __nv_bfloat16 *>(v);
+    auto PK = static_cast<__nv_bfloat16 *>(pk);
+    auto PV = static_cast<__nv_bfloat16 *>(pv);
+    if (L.d == 128)
+        pack_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(L, K, V, idx, PK, PV);
+    else
+        pack_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(L, K, V, idx, PK, PV);
+    return launched();
+}
+
+spava_status run_attn(const Layer &L, const void *q, const void *k, const void *v, const void *pk,
+                      const void *pv, void *o, float *lse, char *ws, cudaStream_t st) {
+    const WsLayout w = ws_layout(L);
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.L = L;
+    SPAVA_TRY(map_tokens(&p.tmQ, q, L, L.Hq));
+    SPAVA_TRY(map_tokens(&p.tmK, k, L, L.Hkv));
+    SPAVA_TRY(map_tokens(&p.tmV, v, L, L.Hkv));
+    // With no packed rows (a = 0, l = 0) no segment reads the packed maps.
+    SPAVA_TRY(L.L > 0 ? map_packed(&p.tmPK, pk, L) : map_tokens(&p.tmPK, k, L, L.Hkv));
+    SPAVA_TRY(L.L > 0 ? map_packed(&p.tmPV, pv, L) : map_tokens(&p.tmPV, v, L, L.Hkv));
+    p.n_groups = plan_attention(L, false, p.groups);
+    p.O = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.part_O = reinterpret_cast<float *>(ws + w.part_o);
+    p.part_lse = reinterpret_cast<float *>(ws + w.part_lse);
+    p.status = reinterpret_cast<int *>(ws + w.status);
+    SPAVA_TRY(L.d == 128 ? launch_attn<128, false>(p, st) : launch_attn<64, false>(p, st));
+    const int64_t warps = static_cast<int64_t>(L.Hq) * L.q;
+    const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+    auto O = static_cast<__nv_bfloat16 *>(o);
+    if (L.d == 128)
+        merge_kernel<128><<<blocks, 256, 0, st>>>(L, p.part_O, p.part_lse, O, lse);
+    else
+        merge_kernel<64><<<blocks, 256, 0, st>>>(L, p.part_O, p.part_lse, O, lse);
+    return launched();
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+spava_status spava_workspace_size(const spava_config *cfg, size_t *bytes) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    if (!bytes) return SPAVA_ERR_INVALID_ARG;
+    *bytes = ws_layout(L).total;
+    return SPAVA_OK;
+}
+
+spava_status spava_packed_len(const spava_config *cfg, int64_t *rows) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    if (!rows) return SPAVA_ERR_INVALID_ARG;
+    *rows = L.L;
+    return SPAVA_OK;
+}
+
+spava_status spava_score(const spava_config *cfg, const void *q, const void *k, float *scores,
+                         void *ws, size_t ws_bytes, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    SPAVA_TRY(check_ptr(q));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(scores));
+    SPAVA_TRY(check_ws(L, ws, ws_bytes));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    SPAVA_TRY(run_stats(L, q, k, static_cast<char *>(ws), st));
+    return run_scores(L, q, k, scores, static_cast<char *>(ws), st);
+}
+
+spava_status spava_topk_select(const spava_config *cfg, const float *scores, int32_t *idx,
+                               void *stream) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    SPAVA_TRY(check_ptr(scores));
+    if (L.l > 0) SPAVA_TRY(check_ptr(idx));
+    return run_topk(L, scores, idx, static_cast<cudaStream_t>(stream));
+}
+
+spava_status spava_pack_passing(const spava_config *cfg, const void *k, const void *v,
+                                const int32_t *idx, void *pk, void *pv, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(v));
+    if (L.l > 0) SPAVA_TRY(check_ptr(idx));
+    if (L.L > 0) {
+        SPAVA_TRY(check_ptr(pk));
+        SPAVA_TRY(check_ptr(pv));
+    }
+    return run_pack(L, k, v, idx, pk, pv, static_cast<cudaStream_t>(stream));
+}
+
+spava_status spava_attn(const spava_config *cfg, const void *q, const void *k, const void *v,
+                        const void *pk, const void *pv, void *o, float *lse, void *ws,
+                        size_t ws_bytes, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    SPAVA_TRY(check_ptr(q));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(v));
+    SPAVA_TRY(check_ptr(o));
+    SPAVA_TRY(check_ptr(lse, false));
+    if (L.L > 0) {
+        SPAVA_TRY(check_ptr(pk));
+        SPAVA_TRY(check_ptr(pv));
+    }
+    SPAVA_TRY(check_ws(L, ws, ws_bytes));
+    return run_attn(L, q, k, v, pk, pv, o, lse, static_cast<char *>(ws),
+                    static_cast<cudaStream_t>(stream));
+}
+
+spava_status spava_prefill_attention(const spava_config *cfg, const void *q, const void *k,
+                                     const void *v, void *o, float *lse, int32_t *idx_out,
+                                     void *ws, size_t ws_bytes, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    SPAVA_TRY(check_ptr(q));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(v));
+    SPAVA_TRY(check_ptr(o));
+    SPAVA_TRY(check_ptr(lse, false));
+    SPAVA_TRY(check_ptr(idx_out, false));
+    SPAVA_TRY(check_ws(L, ws, ws_bytes));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(ws);
+    const WsLayout lay = ws_layout(L);
+    float *scores = reinterpret_cast<float *>(w + lay.scores);
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + lay.idx);
+    void *pk = w + lay.pk;
+    void *pv = w + lay.pv;
+    if (L.n_chunks > 1 && L.l > 0) {
+        SPAVA_TRY(run_stats(L, q, k, w, st));
+        SPAVA_TRY(run_scores(L, q, k, scores, w, st));
+        SPAVA_TRY(run_topk(L, scores, idx, st));
+    }
+    SPAVA_TRY(run_pack(L, k, v, idx, pk, pv, st));
+    return run_attn(L, q, k, v, pk, pv, o, lse, w, st);
+}
+
+spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q_host,
+                                          const void *k_host, const void *v_host, void *o_host,
+                                          float *lse_host, void *q, void *k, void *v, void *o,
+                                          float *lse, void *ws, size_t ws_bytes, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    if (!q_host || !k_host || !v_host || !o_host) return SPAVA_ERR_INVALID_ARG;
+    SPAVA_TRY(check_ptr(q));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(v));
+    SPAVA_TRY(check_ptr(o));
+    SPAVA_TRY(check_ws(L, ws, ws_bytes));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t qb = size_t(L.N) * L.Hq * L.d * 2, kb = size_t(L.N) * L.Hkv * L.d * 2;
+    SPAVA_CUDA(cudaMemcpyAsync(q, q_host, qb, cudaMemcpyHostToDevice, st));
+    SPAVA_CUDA(cudaMemcpyAsync(k, k_host, kb, cudaMemcpyHostToDevice, st));
+    SPAVA_CUDA(cudaMemcpyAsync(v, v_host, kb, cudaMemcpyHostToDevice, st));
+    const bool want_lse = lse && lse_host;
+    SPAVA_TRY(spava_prefill_attention(cfg, q, k, v, o, want_lse ? lse : nullptr, nullptr, ws,
+                                      ws_bytes, stream));
+    SPAVA_CUDA(cudaMemcpyAsync(o_host, o, qb, cudaMemcpyDeviceToHost, st));
+    if (want_lse)
+        SPAVA_CUDA(cudaMemcpyAsync(lse_host, lse, sizeof(float) * size_t(L.Hq) * L.N,
+                                   cudaMemcpyDeviceToHost, st));
+    return SPAVA_OK;
+}
+
+spava_status spava_device_status(void *ws, size_t ws_bytes, void *stream, int32_t *flags) {
+    if (!ws || ws_bytes < 256 || !flags) return SPAVA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    SPAVA_CUDA(cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st));
+    SPAVA_CUDA(cudaStreamSynchronize(st));
+    if (h) {
+        SPAVA_CUDA(cudaMemsetAsync(ws, 0, sizeof(h), st));
+        SPAVA_CUDA(cudaStreamSynchronize(st));
+    }
+    *flags = h;
+    return (h & kStatusTimeout) ? SPAVA_ERR_TIMEOUT : SPAVA_OK;
+}
+
+spava_status spava_attended_pairs(const spava_config *cfg, int64_t pairs[3], int64_t *per_host) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    if (!pairs) return SPAVA_ERR_INVALID_ARG;
+    pairs[0] = pairs[1] = pairs[2] = 0;
+    if (per_host)
+        for (int p = 0; p < L.H; ++p) per_host[p] = 0;
+    Group groups[sizeof(AttnParams::groups) / sizeof(Group)];
+    const int ng = plan_attention(L, false, groups);
+    for (int k = 0; k < ng; ++k) {
+        for (int rt = 0; rt < groups[k].n_rt; ++rt) {
+            Item it{groups[k].kind, groups[k].sub, rt, 0};
+            Seg s[kMaxSegs];
+            const int n = build_segments(L, it, s);
+            int row0, row_end;
+            item_rows(L, it, row0, row_end);
+            int64_t cnt = 0;
+            for (int t = row0; t < row_end; ++t)
+                for (int i = 0; i < n; ++i) {
+                    const int e = s[i].causal ? std::min(s[i].end, t + 1) : s[i].end;
+                    cnt += std::max(0, e - s[i].begin);
+                }
+            const int cls = it.kind == kAnchor ? 0 : it.kind == kCtx ? 1 : 2;
+            pairs[cls] += cnt;
+            if (per_host && it.kind == kCtx) per_host[pair_of(L.H, it.sub)] += cnt;
+        }
+    }
+    return SPAVA_OK;
+}
+
+const char *spava_status_string(spava_status s) {
+    switch (s) {
+        case SPAVA_OK: return "ok";
+        case SPAVA_ERR_INVALID_ARG: return "invalid argument";
+        case SPAVA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case SPAVA_ERR_MISALIGNED: return "misaligned pointer";
+        case SPAVA_ERR_WORKSPACE: return "workspace missing or too small";
+        case SPAVA_ERR_CUDA: return "CUDA error";
+        case SPAVA_ERR_TIMEOUT: return "kernel wait timed out";
+    }
+    return "unknown status";
+}
+
+int32_t spava_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

@@ -1,0 +1,173 @@
+"""GPU parity of every step of the path against the fp64 oracle, element by
+element, on sizes the oracle finishes in seconds that still span several 128
+tiles and ragged tails (chunk, anchor and query lengths not multiples of 128,
+GQA groups of 2 and 7, d = 64 and 128, uneven chunks, a = 0, one host, full
+passing blocks, local_pair_full = 0)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import (LSE_ABS, SCORE_REL, OracleRun, check_outputs, check_selection, to_np)
+from sequence_sparse_attention_b200.api import Layout, Spava
+from sequence_sparse_attention_b200.synth import WORKLOADS, Workload, chunk_offsets, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": WORKLOADS["tiny"],
+    "g7": Workload("g7", H=2, Hq=14, Hkv=2, d=128, N=1500, a=100, q=150, l=100, frame=32, seed=11),
+    "g7_pure": Workload("g7_pure", H=2, Hq=14, Hkv=2, d=128, N=1500, a=100, q=150, l=100, frame=32,
+                        seed=11, local_pair_full=0),
+    "no_anchor": Workload("no_anchor", H=3, Hq=8, Hkv=4, d=128, N=1300, a=0, q=64, l=64, frame=32,
+                          seed=12),
+    "one_host": Workload("one_host", H=1, Hq=4, Hkv=2, d=128, N=1000, a=64, q=40, l=30, frame=32,
+                         seed=13),
+    "full_l": Workload("full_l", H=3, Hq=4, Hkv=1, d=64, N=1200, a=200, q=130, l=100000, frame=32,
+                       seed=14),
+    "jitter_heavy": Workload("jitter_heavy", H=3, Hq=6, Hkv=2, d=64, N=64 * 30 + 70 + 90, a=70, q=90,
+                             l=45, frame=64, jitter=0.1, heavy_frac=0.05, seed=15),
+    "long_anchor": Workload("long_anchor", H=2, Hq=4, Hkv=4, d=128, N=1800, a=300, q=257, l=160,
+                            frame=32, seed=16),
+}
+
+_cache = {}
+
+
+def setup_case(name):
+    if name not in _cache:
+        w = CASES[name]
+        Q, K, V, off = make_inputs(w)          # CPU generator, copied to the GPU below
+        ref = OracleRun(w, Q, K, V)
+        rows = np.arange(w.N)
+        O_ref, lse_ref = ref.rows(rows, list(range(w.Hq)))
+        _cache[name] = (w, Q, K, V, ref, O_ref, lse_ref)
+    return _cache[name]
+
+
+def device_clean(sp: Spava):
+    assert sp.device_status() == 0, "a kernel wait timed out"
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_scores(name):
+    w, Q, K, V, ref, _, _ = setup_case(name)
+    sp = Spava(Layout.from_workload(w))
+    scores = to_np(sp.score(Q.cuda(), K.cuda()))
+    device_clean(sp)
+    off = chunk_offsets(w)
+    G = w.Hq // w.Hkv
+    last0 = int(off[-2] - w.a)          # the last chunk produces no passing block
+    want = ref.scores[:, :last0]
+    got = scores[:, :last0]
+    np.testing.assert_allclose(got, want, rtol=SCORE_REL, atol=1e-7 * G * w.q)
+    for u in range(2 * w.H - 1):        # closed form: each chunk's scores sum to G*q
+        s0, s1 = int(off[u] - w.a), int(off[u + 1] - w.a)
+        np.testing.assert_allclose(got[:, s0:s1].sum(axis=1), G * w.q, rtol=1e-4)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_topk_bit_exact_on_fp32_scores(name):
+    """Selection from the same fp32 scores: index sets bit-exact (ties to the
+    lower index), against the oracle's sort run on those fp32 values."""
+    w, Q, K, V, ref, _, _ = setup_case(name)
+    sp = Spava(Layout.from_workload(w))
+    off = chunk_offsets(w)
+    s32 = ref.scores.astype(np.float32)
+    # plant exact ties across a chunk so the tie rule decides
+    s32[:, 5:40] = s32[:, 3:4]
+    idx = to_np(sp.topk_select(torch.from_numpy(s32).cuda())).astype(np.int32)
+    for u in range(2 * w.H - 1):
+        s0 = int(off[u] - w.a)
+        n = int(off[u + 1] - off[u])
+        for g in range(w.Hkv):
+            want = oracle.select_top_l(s32[g, s0:s0 + n].astype(np.float64), int(off[u]), w.l)
+            np.testing.assert_array_equal(idx[u, g], want, err_msg=f"{name} u={u} g={g}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "g7", "no_anchor", "long_anchor"])
+def test_pack_exact(name):
+    w, Q, K, V, ref, _, _ = setup_case(name)
+    sp = Spava(Layout.from_workload(w))
+    Kd, Vd = K.cuda(), V.cuda()
+    idx = torch.from_numpy(ref.idx).cuda()
+    pk, pv = sp.pack_passing(Kd, Vd, idx)
+    torch.cuda.synchronize()
+    off = chunk_offsets(w)
+    for g in range(w.Hkv):
+        rows = list(range(w.a))
+        for u in range(2 * w.H - 1):
+            k = min(w.l, int(off[u + 1] - off[u]))
+            rows += ref.idx[u, g, :k].tolist()
+        r = torch.tensor(rows, dtype=torch.long)
+        assert torch.equal(pk[g].cpu().view(torch.int16), K[r, g].view(torch.int16))
+        assert torch.equal(pv[g].cpu().view(torch.int16), V[r, g].view(torch.int16))
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_attn_given_oracle_selection(name):
+    """spava_attn on passing blocks packed from the oracle's own selection:
+    every row and head against the oracle."""
+    w, Q, K, V, ref, O_ref, lse_ref = setup_case(name)
+    sp = Spava(Layout.from_workload(w))
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    pk, pv = sp.pack_passing(Kd, Vd, torch.from_numpy(ref.idx).cuda())
+    O, lse = sp.attn(Qd, Kd, Vd, pk, pv)
+    device_clean(sp)
+    check_outputs(to_np(O), O_ref, name)
+    np.testing.assert_allclose(to_np(lse).T, lse_ref, atol=LSE_ABS, rtol=0)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_end_to_end(name):
+    w, Q, K, V, ref, O_ref, lse_ref = setup_case(name)
+    sp = Spava(Layout.from_workload(w))
+    O, lse, idx = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda(), want_idx=True)
+    device_clean(sp)
+    check_selection(w, ref.scores, idx.cpu().numpy(), range(w.Hkv))
+    check_outputs(to_np(O), O_ref, name)
+    np.testing.assert_allclose(to_np(lse).T, lse_ref, atol=LSE_ABS, rtol=0)
+
+
+def test_values_one_give_ones():
+    """V = 1 everywhere: every softmax-weighted average is exactly one up to
+    the bf16 rounding of P."""
+    w = CASES["g7"]
+    Q, K, V, _ = make_inputs(w)
+    V = torch.ones_like(V)
+    sp = Spava(Layout.from_workload(w))
+    O, _, _ = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda())
+    device_clean(sp)
+    err = (O.float() - 1).abs()
+    assert err.max().item() < 1e-2 and err.mean().item() < 2e-3
+
+
+def test_repeat_calls_bit_identical():
+    w = CASES["g7"]
+    Q, K, V, _ = make_inputs(w)
+    sp = Spava(Layout.from_workload(w))
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    O1, l1, i1 = sp.prefill_attention(Qd, Kd, Vd, want_idx=True)
+    O2, l2, i2 = sp.prefill_attention(Qd, Kd, Vd, want_idx=True)
+    device_clean(sp)
+    assert torch.equal(i1, i2)
+    assert torch.equal(O1.view(torch.int16), O2.view(torch.int16))
+    assert torch.equal(l1, l2)
+
+
+def test_host_buffers_entry_point():
+    w = CASES["tiny"]
+    Q, K, V, _ = make_inputs(w)
+    sp = Spava(Layout.from_workload(w))
+    qh, kh, vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
+    oh = torch.empty_like(Q).pin_memory()
+    lh = torch.empty((w.Hq, w.N), dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(Q, device="cuda"), torch.empty_like(K, device="cuda"), torch.empty_like(V, device="cuda")
+    od = torch.empty_like(qd)
+    ld = torch.empty((w.Hq, w.N), dtype=torch.float32, device="cuda")
+    sp.prefill_attention_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld)
+    torch.cuda.synchronize()
+    device_clean(sp)
+    O_dev, lse_dev, _ = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda())
+    assert torch.equal(oh.view(torch.int16), O_dev.cpu().view(torch.int16))
+    assert torch.equal(lh, lse_dev.cpu())
