@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Throughput of the approximate-attention prefill layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 128k] [--impl ours|reference]
+
+One step = one pass of the whole path over one layer: query-block scores
+(statistics + scoring kernels), top-l selection, passing-block gather, and the
+approximate attention with the query-row merge -- the libspava C ABI calls
+spava_score -> spava_topk_select -> spava_pack_passing -> spava_attn, on inputs
+resident in HBM.  Prints one JSON line (rank 0).
+
+Multi-GPU: each rank runs its own independent layer (weak scaling, no data
+collective); the process group only provides the barrier and the max-over-ranks
+timing.  ``--impl reference`` times the fp64 CPU oracle on a bounded sample of
+the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sequence_sparse_attention_b200.api import Layout, Spava, attended_pairs  # noqa: E402
+from sequence_sparse_attention_b200.synth import WORKLOADS, chunk_offsets, make_inputs  # noqa: E402
+
+METRIC = "approx-attn prefill tokens/s per layer on 1 B200; % BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 6   # stats, scores, top-l, pack, attention, query merge
+
+# DRAM traffic of one attention launch from an ncu capture (profiles/), valid
+# only while the kernel source is unchanged (sha256 of attn_kernel.cuh).
+PROFILED_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None, "source": None}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sha() -> str:
+    p = os.path.join(ROOT, "sequence_sparse_attention_b200", "csrc", "attn_kernel.cuh")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+def physical_gpu(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x for x in vis.split(",") if x.strip()]
+    if local < len(ids) and ids[local].strip().isdigit():
+        return int(ids[local])
+    return local
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------- oracle
+def oracle_inputs(w, Q=None, K=None, V=None):
+    """Host bf16 bit patterns of the layer's inputs (the given tensors, or a
+    fresh CPU draw of the same workload)."""
+    from sequence_sparse_attention_b200.synth import bf16_bits
+    if Q is None:
+        Q, K, V, _ = make_inputs(w)
+    return bf16_bits(Q), bf16_bits(K), bf16_bits(V)
+
+
+def oracle_sample(w, budget_s: float, inputs, seed: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload and extrapolate
+    to one whole layer.  Returns (tokens/s, description, threads, seconds)."""
+    import oracle
+    Qb, Kb, Vb = inputs
+    off = chunk_offsets(w)
+    p = oracle.Problem(H=w.H, Hq=w.Hq, Hkv=w.Hkv, d=w.d, N=w.N, a=w.a, q=w.q, offsets=off,
+                       l=w.l, local_pair_full=w.local_pair_full)
+    G = w.Hq // w.Hkv
+    # (1) scores of chunk 0, KV head 0, and their selection
+    t0 = time.perf_counter()
+    S = oracle.chunk_scores(p, Qb, Kb, 0, 0)
+    t_score = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.select_top_l(S, int(off[0]), w.l)
+    t_select = time.perf_counter() - t0
+    n0 = int(off[1] - off[0])
+    scored_total = sum(int(off[u + 1] - off[u]) for u in range(2 * w.H - 1)) * w.Hkv
+    # (2) attention rows of the heads of KV group 0, spread over the sequence
+    idx = np.full((2 * w.H - 1, w.Hkv, w.l), -1, dtype=np.int32)
+    for u in range(2 * w.H - 1):
+        k = min(w.l, int(off[u + 1] - off[u]))
+        idx[u, :, :k] = off[u] + np.arange(k)       # any valid selection costs the same
+    rng = np.random.default_rng(seed)
+    rows_all = rng.permutation(w.N)
+    heads = list(range(G))
+    done_rows, pairs, t_attn = 0, 0, 0.0
+    remaining = max(1.0, budget_s - t_score - t_select)
+    batch = 8
+    while t_attn < remaining and done_rows < len(rows_all):
+        rows = rows_all[done_rows:done_rows + batch]
+        t0 = time.perf_counter()
+        oracle.prefill_rows(p, Qb, Kb, Vb, idx, rows, heads)
+        t_attn += time.perf_counter() - t0
+        pairs += sum(len(oracle.key_set(p, idx, int(t), 0)) for t in rows) * G
+        done_rows += len(rows)
+        batch = min(64, batch * 2)
+    total_pairs = sum(attended_pairs(Layout.from_workload(w))[0]) * w.Hq
+    t_layer = (t_score * scored_total / n0 + t_select * (2 * w.H - 1) * w.Hkv
+               + t_attn * total_pairs / pairs)
+    desc = (f"scores of chunk 0 for KV head 0 ({n0} keys x {G * w.q} query rows) and its top-l; "
+            f"attention of {done_rows} random rows x {G} heads ({pairs} pairs); extrapolated to the "
+            f"layer by scored keys and attended pairs; {t_score + t_select + t_attn:.1f} s of CPU")
+    return w.N / t_layer, desc, oracle.num_threads(), t_score + t_select + t_attn
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    values, cores, desc, spent = [], None, None, 0.0
+    per_step = max(3.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    inputs = oracle_inputs(w)
+    for s in range(args.warmup + args.steps):
+        v, desc, cores, sp = oracle_sample(w, per_step, inputs, seed=s)
+        spent += sp
+        if s >= args.warmup:
+            values.append(v)
+    value = statistics.median(values)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * w.N / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": f"{w.name}: H={w.H} ({2 * w.H} ZigZag virtual hosts), {w.Hq} q / {w.Hkv} kv heads, "
+                        f"d={w.d}, {w.N} tokens (anchor {w.a}, query block {w.q}), top-l={w.l}",
+            "tokens": w.N, "H": w.H, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
+            "anchor": w.a, "query_block": w.q, "top_l": w.l,
+            "local_pair_full": w.local_pair_full,
+            "inputs": "seeded synthetic video-shaped bf16 (frame-correlated keys"
+                      + (", 5% heavy-hitter keys" if w.heavy_frac else "")
+                      + (", +/-10% uneven chunks" if w.jitter else "") + ")",
+            "l2": "no flush: inputs (Q+K+V) exceed the 126 MB L2"}
+
+
+# ----------------------------------------------------------------------- ours
+def run_ours(args, world, rank, local):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = WORKLOADS[args.workload]
+    Q, K, V, off = make_inputs(w, device)
+    lay = Layout.from_workload(w)
+    sp = Spava(lay, device)
+    scores = torch.zeros((w.Hkv, lay.context), dtype=torch.float32, device=device)
+    idx = torch.empty((2 * w.H - 1, w.Hkv, w.l), dtype=torch.int32, device=device)
+    pk = torch.empty((w.Hkv, sp.L, w.d), dtype=torch.bfloat16, device=device)
+    pv = torch.empty_like(pk)
+    O = torch.empty_like(Q)
+    lse = torch.empty((w.Hq, w.N), dtype=torch.float32, device=device)
+
+    def step(ev=None):
+        if ev: ev[0].record()
+        sp.score(Q, K, scores)
+        if ev: ev[1].record()
+        sp.topk_select(scores, idx)
+        if ev: ev[2].record()
+        sp.pack_passing(K, V, idx, pk, pv)
+        if ev: ev[3].record()
+        sp.attn(Q, K, V, pk, pv, O, lse)
+        if ev: ev[4].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = sp.device_status()
+    if status:
+        raise RuntimeError(f"kernel status {status} during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(physical_gpu(local))
+    with sampler:
+        time.sleep(0.3)
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record()
+        for s in range(args.steps):
+            step(evs[s])
+        end.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    clocks = sampler.summary()
+    if sp.device_status():
+        raise RuntimeError("kernel status set during the timed region")
+    ms_total = max_over_ranks(start.elapsed_time(end), world)
+    names = ["score", "topk", "pack", "attn"]
+    per = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
+           for i, n in enumerate(names)}
+    ms_step = ms_total / args.steps
+    tokens_per_s = world * w.N * args.steps / (ms_total / 1e3)
+
+    # ---- roofline of the dominant kernel (approximate attention)
+    pk_, pe = peaks()
+    pairs = sum(attended_pairs(lay)[0])
+    flops = 4.0 * w.d * w.Hq * pairs
+    achieved = flops / (per["attn"] / 1e3) / 1e12
+    peak = pk_.get("bf16_tflops_sustained") or pk_.get("bf16_tflops")
+    traffic = None
+    if PROFILED_TRAFFIC["kernel_sha256"] == kernel_sha():
+        traffic = PROFILED_TRAFFIC["bytes_per_launch"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": "attn_kernel<128,false> + query merge (spava_attn)",
+                "peak_kind": f"{pe} bf16 dense, sustained (kernel timed inside a long step)",
+                "frac_of_burst_peak": achieved / pk_.get("bf16_tflops", peak),
+                "algorithmic_flops_per_launch": flops, "attended_pairs_per_head": pairs}
+
+    # ---- end to end through the host-buffer entry point
+    qh = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+    kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
+    vh = torch.empty(V.shape, dtype=V.dtype, pin_memory=True)
+    qh.copy_(Q)
+    kh.copy_(K)
+    vh.copy_(V)
+    oh = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    sp.prefill_attention_host(qh, kh, vh, oh, None, Q, K, V, O, None)  # warm
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        sp.prefill_attention_host(qh, kh, vh, oh, None, Q, K, V, O, None)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = (Q.numel() + K.numel() + V.numel()) * 2
+    d2h = O.numel() * 2
+    e2e = {"value": world * w.N / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+           "api": "spava_prefill_attention_host (pinned host buffers in/out)"}
+
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(w),
+        "roofline": roofline,
+        "kernel_ms": per,
+        "tensor_peak_frac": {"of_sustained": achieved / peak,
+                             "of_burst": achieved / pk_.get("bf16_tflops", peak),
+                             "of_nominal_2250": achieved / 2250.0},
+        "e2e": e2e, "gpu_launches": KERNELS_PER_STEP * args.steps, "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, cores, _ = oracle_sample(w, args.cpu_budget, oracle_inputs(w, Q, K, V))
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="128k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
