@@ -153,6 +153,29 @@ spava_status spava_device_status(void *ws, size_t ws_bytes, void *stream, int32_
  * "Bilanciamento del Carico dell'Attenzione Approssimata").  Host only. */
 spava_status spava_attended_pairs(const spava_config *cfg, int64_t pairs[3], int64_t *per_host);
 
+/* spava_score for callers that cannot allocate device memory: same inputs,
+ * same scores output, no workspace argument.  (The pages have no counterpart:
+ * this is an interface choice of the library, not part of the method.)
+ * Who needs it: code that is handed only its input and output buffers, such
+ * as a plug-in inside an engine that owns all device memory, or code that must
+ * not allocate after start-up (real-time or certified deployments, or a
+ * latency-critical path where cudaMalloc would synchronise the device).
+ * The scratch for the per-chunk softmax statistics is a fixed 4 MiB array
+ * compiled into the library (each GPU that loads the library holds it until
+ * the process exits).  Limit: 256 + 4*(2H-1)*Hq*q bytes must fit in 4 MiB
+ * (e.g. H=16, Hq=32, q=512 needs 2 MiB); larger layers get
+ * SPAVA_ERR_WORKSPACE and nothing is launched.  No allocation of any kind
+ * (no cudaMalloc, cudaFree or allocating library routine).
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * All calls share the one array: calls that overlap on the GPU (other streams,
+ * other host threads) race and must be serialised by the caller.  A kernel
+ * wait that gives up is recorded in the array's status word, which each call
+ * clears at its start; it is not reported to the caller (use spava_score with
+ * a workspace and spava_device_status where that matters). */
+spava_status spava_score_noalloc(const spava_config *cfg, const void *q, const void *k,
+                                 float *scores, void *stream);
+
 const char *spava_status_string(spava_status s);
 
 /* The CUDA error code of this thread's last SPAVA_ERR_CUDA (0 if none). */

@@ -519,3 +519,99 @@ const char *spava_status_string(spava_status s) {
 int32_t spava_last_cuda_error(void) { return g_last_cuda_error; }
 
 }  // extern "C"
+
+// ==================================================================== scores
+// without caller-provided scratch
+//
+// spava_score needs scratch memory for the per-chunk softmax statistics of the
+// query block, which normally lives in the caller's workspace.  Some callers
+// cannot provide one: a plug-in inside a host engine that owns all device
+// memory and hands a kernel only its input and output buffers, or code that
+// must not allocate after start-up (real-time or certified deployments, and
+// latency-critical paths where cudaMalloc would synchronise the device).  For
+// them the scratch lives in the fixed array below, compiled into the library:
+// every GPU that loads the library holds these bytes until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr size_t kNoAllocStatusBytes = 256;                // status word, then statistics
+
+static __device__ __align__(256) unsigned char g_score_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_score_scratch on the current device.  The name is only
+// a host-side stand-in for the array, so the address is looked up once per
+// device, with that device current.
+spava_status scratch_address(void **out) {
+    int dev = 0;
+    SPAVA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return SPAVA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        SPAVA_CUDA(cudaGetSymbolAddress(&p, g_score_scratch));
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return SPAVA_OK;
+}
+
+}  // namespace
+
+extern "C" spava_status spava_score_noalloc(const spava_config *cfg, const void *q, const void *k,
+                                            float *scores, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_layer(cfg, &L));
+    SPAVA_TRY(check_ptr(q));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(scores));
+    const size_t stats_bytes = sizeof(float) * size_t(L.n_chunks - 1) * L.Hq * L.q;
+    if (kNoAllocStatusBytes + stats_bytes > kNoAllocScratchBytes) return SPAVA_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    SPAVA_TRY(scratch_address(&scratch));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *base = static_cast<char *>(scratch);
+    int *status = reinterpret_cast<int *>(base);
+    float *stats = reinterpret_cast<float *>(base + kNoAllocStatusBytes);
+    // The array keeps the previous call's contents: the status word must start
+    // at zero; every statistic is written before it is read.
+    SPAVA_CUDA(cudaMemsetAsync(status, 0, sizeof(int), st));
+
+    AttnParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.L = L;
+    SPAVA_TRY(map_tokens(&sp.tmQ, q, L, L.Hq));
+    SPAVA_TRY(map_tokens(&sp.tmK, k, L, L.Hkv));
+    sp.n_groups = plan_attention(L, true, sp.groups);
+    sp.stats = stats;
+    sp.status = status;
+    SPAVA_TRY(L.d == 128 ? launch_attn<128, true>(sp, st) : launch_attn<64, true>(sp, st));
+
+    ScoreParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.L = L;
+    p.tmQ = sp.tmQ;
+    p.tmK = sp.tmK;
+    p.stats = stats;
+    p.scores = scores;
+    p.status = status;
+    int tiles = 0;
+    for (int u = 0; u < L.n_chunks - 1; ++u) {
+        p.tile_begin[u] = tiles;
+        tiles += cdiv(L.off[u + 1] - L.off[u], 128);
+    }
+    p.tile_begin[L.n_chunks - 1] = tiles;
+    const int64_t blocks = static_cast<int64_t>(tiles) * L.Hkv;
+    if (blocks == 0) return SPAVA_OK;
+    if (L.d == 128) {
+        SPAVA_TRY(set_smem(score_kernel<128>, ScoreSmem<128>::kAlloc));
+        score_kernel<128><<<static_cast<unsigned>(blocks), 192, ScoreSmem<128>::kAlloc, st>>>(p);
+    } else {
+        SPAVA_TRY(set_smem(score_kernel<64>, ScoreSmem<64>::kAlloc));
+        score_kernel<64><<<static_cast<unsigned>(blocks), 192, ScoreSmem<64>::kAlloc, st>>>(p);
+    }
+    return launched();
+}
