@@ -140,6 +140,19 @@ __host__ __device__ inline int build_segments(const Layer &L, const Item &it, Se
     return n;
 }
 
+// Position in an item's key sequence: segment index and 128-key tile inside it.
+struct TileCursor {
+    int seg = 0, tile = 0;
+    __host__ __device__ void advance(const Seg *s) {
+        if (s[seg].begin + (tile + 1) * kKeyTile >= s[seg].end) {
+            ++seg;
+            tile = 0;
+        } else {
+            ++tile;
+        }
+    }
+};
+
 __host__ __device__ inline int count_tiles(const Seg *s, int n) {
     int t = 0;
     for (int i = 0; i < n; ++i) t += cdiv(s[i].end - s[i].begin, kKeyTile);

@@ -45,6 +45,8 @@ struct ScoreSmem {
     static constexpr int kAlloc = kBytes + 1024;
 };
 
+static_assert(ScoreSmem<128>::kAlloc <= 232448, "scoring smem over budget");
+
 template <int D>
 __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ ScoreParams P) {
     using SM = ScoreSmem<D>;
@@ -153,7 +155,9 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ S
         const int j = threadIdx.x;  // key within the tile == TMEM lane
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const float sl2 = L.scale_log2;
-        float acc = 0.f;
+        float2 acc[4];  // 8 independent partial sums, in packed pairs
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
         bool ok = true;
         for (int b = 0; b < NBLK; ++b) {
             const int sb = b % NB;
@@ -166,28 +170,29 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ S
             tc_fence_after();
             float x[128];
             {
-                uint32_t r[32];
+                uint32_t r[128];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(lane_addr + sb * 128 + c * 32, r);
-                    tmem_wait_ld();
+                for (int c = 0; c < 4; ++c)
+                    tmem_ld32(lane_addr + sb * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+                tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
-                }
+                for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(r[e]);
             }
             tc_fence_before();
             mbar_arrive(&s_free[sb]);
-            if (n_rows == 128) {
+            const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-                for (int c = 0; c < 128; ++c) acc += ex2(fmaf(x[c], sl2, -__ldg(lse2 + c)));
-            } else {
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c < n_rows) acc += ex2(fmaf(x[c], sl2, -__ldg(lse2 + c)));
+            for (int c = 0; c < 128; c += 2) {
+                const float2 nl = make_float2(c < n_rows ? -__ldg(lse2 + c) : -INFINITY,
+                                              c + 1 < n_rows ? -__ldg(lse2 + c + 1) : -INFINITY);
+                const float2 arg = ffma2(make_float2(x[c], x[c + 1]), sl2v, nl);
+                acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(arg.x), ex2(arg.y)));
             }
         }
         if (ok && j < n_valid)
-            P.scores[static_cast<size_t>(g) * L.C + (key0 - L.a) + j] = acc;
+            P.scores[static_cast<size_t>(g) * L.C + (key0 - L.a) + j] =
+                ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
     }
 
     tc_fence_before();

@@ -160,6 +160,37 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// Four MMAs in one asm block: D (+)= A_k B_k, k = 0..3.  The first one
+// accumulates only if acc0 != 0, the rest always.  Grouping keeps the issuing
+// thread to one instruction per MMA, so it is not slowed by busy warps that
+// share its scheduler.
+__device__ __forceinline__ void mma_ss_x4(uint32_t d_tmem, uint64_t a0, uint64_t a1, uint64_t a2,
+                                          uint64_t a3, uint64_t b0, uint64_t b1, uint64_t b2,
+                                          uint64_t b3, uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t"
+        "setp.ne.b32 p0, %10, 0;\n\tsetp.eq.b32 p1, %10, %10;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %1, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %1, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %1, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %9, %1, p1;\n\t}\n" ::"r"(d_tmem),
+        "r"(idesc), "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3),
+        "r"(acc0));
+}
+__device__ __forceinline__ void mma_ts_x4(uint32_t d_tmem, uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint64_t b0, uint64_t b1, uint64_t b2,
+                                          uint64_t b3, uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t"
+        "setp.ne.b32 p0, %10, 0;\n\tsetp.eq.b32 p1, %10, %10;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %1, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %1, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %1, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %9, %1, p1;\n\t}\n" ::"r"(d_tmem),
+        "r"(idesc), "r"(a0), "r"(a1), "r"(a2), "r"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3),
+        "r"(acc0));
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane
 // (32*(warp%4) + i) of the given columns.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -193,6 +224,23 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ named barriers
+__device__ __forceinline__ void bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Named barrier that also ANDs a predicate over its participants: every
+// participant gets the same answer, so they can leave a loop together.
+__device__ __forceinline__ bool bar_red_and(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
 // ------------------------------------------------------------------ math
 // Hardware base-2 exponential (MUFU.EX2), flush-to-zero approximate.
 __device__ __forceinline__ float ex2(float x) {
@@ -200,6 +248,45 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of work,
+// which also keeps the issue port free for the MMA-issuing thread.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// Max of 64 values with 4 independent chains of 3-input max.
+__device__ __forceinline__ float max64(const float (&x)[64]) {
+    float m[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = x[k];
+#pragma unroll
+    for (int c = 4; c + 8 <= 64; c += 8)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m[k] = fmax3(m[k], x[c + k], x[c + 4 + k]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], x[60 + k]);
+    return fmaxf(fmax3(m[0], m[1], m[2]), m[3]);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
     return *reinterpret_cast<uint32_t *>(&v);

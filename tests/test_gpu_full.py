@@ -1,0 +1,70 @@
+"""Parity at the full layer sizes of the long-video study (16K, 64K, 128K and
+256K tokens), in the launch configuration bench.py times (the four C-ABI steps
+on one stream), checked on what the oracle can compute one by one: the scores
+and passing blocks of sampled KV groups, and the outputs of sampled rows
+(first/last rows of every chunk and of every 128-row tile edge, random rows,
+anchor and query rows) for every query head of those groups.  Every selection
+of every group is also checked for validity (ascending, inside its chunk,
+-1 padded)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import (LSE_ABS, SCORE_REL, check_outputs, check_selection, problem, sample_rows,
+                         to_np)
+from sequence_sparse_attention_b200.api import Layout, Spava
+from sequence_sparse_attention_b200.synth import WORKLOADS, bf16_bits, chunk_offsets, make_inputs
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def run_layer_like_bench(sp: Spava, Q, K, V):
+    w = sp.lay
+    scores = torch.zeros((w.Hkv, w.context), dtype=torch.float32, device=Q.device)
+    idx = torch.empty((2 * w.H - 1, w.Hkv, w.l), dtype=torch.int32, device=Q.device)
+    sp.score(Q, K, scores)
+    sp.topk_select(scores, idx)
+    pk, pv = sp.pack_passing(K, V, idx)
+    O, lse = sp.attn(Q, K, V, pk, pv)
+    torch.cuda.synchronize()
+    return scores, idx, O, lse
+
+
+@pytest.mark.parametrize("name", ["16k", "64k", "128k", "256k"])
+def test_full_size_layer(name):
+    w = WORKLOADS[name]
+    Q, K, V, off = make_inputs(w, "cuda")
+    sp = Spava(Layout.from_workload(w))
+    scores, idx, O, lse = run_layer_like_bench(sp, Q, K, V)
+    assert sp.device_status() == 0
+    idx_h = idx.cpu().numpy()
+
+    # every selection is well formed
+    for u in range(2 * w.H - 1):
+        k = min(w.l, int(off[u + 1] - off[u]))
+        sel = idx_h[u, :, :k]
+        assert (np.diff(sel, axis=1) > 0).all()
+        assert ((sel >= off[u]) & (sel < off[u + 1])).all()
+        assert (idx_h[u, :, k:] == -1).all()
+
+    groups = sorted({0, w.Hkv - 1})
+    p = problem(w, off)
+    Qb, Kb, Vb = bf16_bits(Q), bf16_bits(K), bf16_bits(V)
+    sc_ref, idx_ref = oracle.scores_and_select(p, Qb, Kb, groups)
+    sc = to_np(scores)
+    last0 = int(off[-2] - w.a)
+    for g in groups:
+        np.testing.assert_allclose(sc[g, :last0], sc_ref[g, :last0], rtol=SCORE_REL,
+                                   atol=1e-7 * w.q * w.Hq / w.Hkv)
+    n_exact, n_band = check_selection(w, sc_ref, idx_h, groups)
+
+    G = w.Hq // w.Hkv
+    heads = [h for g in groups for h in range(g * G, (g + 1) * G)]
+    rows = sample_rows(w, per_chunk=8, seed=1)
+    O_ref, lse_ref = oracle.prefill_rows(p, Qb, Kb, Vb, idx_ref, rows, heads)
+    O_got = to_np(O[torch.from_numpy(rows).cuda()][:, heads])
+    mx, mean = check_outputs(O_got, O_ref, name)
+    lse_got = to_np(lse[heads][:, torch.from_numpy(rows).cuda()]).T
+    np.testing.assert_allclose(lse_got, lse_ref, atol=LSE_ABS, rtol=0)
+    print(f"{name}: selections exact {n_exact}, in-band {n_band}; O max {mx:.2e} mean {mean:.2e}")
