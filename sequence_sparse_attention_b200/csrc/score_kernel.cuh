@@ -30,6 +30,12 @@ struct ScoreParams {
     int32_t tile_begin[kMaxChunks + 1];  // prefix of 128-key tiles over chunks u < 2H-1
 };
 
+constexpr int kScoreWarps = 16;                 // 4 per TMEM lane quarter
+constexpr int kScoreThreads = kScoreWarps * 32;
+constexpr int kScoreProducer = kScoreWarps;
+constexpr int kScoreMma = kScoreWarps + 1;
+constexpr int kScoreBlockThreads = (kScoreWarps + 2) * 32;
+
 template <int D>
 struct ScoreSmem {
     static constexpr int kPanels = D / 64;
@@ -40,7 +46,8 @@ struct ScoreSmem {
     static constexpr int kOffQ = kTile;
     static constexpr int kOffBar = kOffQ + QS * kTile;
     static constexpr int kNumBar = 1 + 2 * QS + 2 * NB + 1;
-    static constexpr int kOffMisc = kOffBar + kNumBar * 8;
+    static constexpr int kOffRed = kOffBar + kNumBar * 8;   // [4 parts][128 keys] partial sums
+    static constexpr int kOffMisc = kOffRed + 4 * 128 * 4;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
 };
@@ -48,7 +55,7 @@ struct ScoreSmem {
 static_assert(ScoreSmem<128>::kAlloc <= 232448, "scoring smem over budget");
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ ScoreParams P) {
+__global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __grid_constant__ ScoreParams P) {
     using SM = ScoreSmem<D>;
     constexpr int QS = SM::QS, NB = SM::NB;
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, 0, 0);
@@ -87,24 +94,24 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ S
         }
         for (int i = 0; i < NB; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 128);
+            mbar_init(&s_free[i], kScoreThreads);
         }
         mbar_init(mma_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == kScoreProducer && lane == 0) {
         tma_prefetch(&P.tmQ);
         tma_prefetch(&P.tmK);
     }
-    if (warp == 5) tmem_alloc(tmem_slot, 512);
+    if (warp == kScoreMma) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const AbortState ab{abort_flag, P.status};
 
-    if (warp == 4) {
+    if (warp == kScoreProducer) {
         if (lane == 0) {
             mbar_expect_tx(a_full, SM::kTile);
             for (int p = 0; p < SM::kPanels; ++p)
@@ -126,7 +133,7 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ S
             for (int i = 0; i < QS; ++i)
                 if (q_last[i] >= 0) mbar_wait_drain(&q_full[i], (q_last[i] / QS) & 1);
         }
-    } else if (warp == 5) {
+    } else if (warp == kScoreMma) {
         if (lane == 0) {
             const uint32_t a_base = smem_u32(smem + SM::kOffK);
             const uint32_t q_base = smem_u32(smem + SM::kOffQ);
@@ -152,9 +159,13 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ S
         }
         __syncwarp();
     } else {
-        const int j = threadIdx.x;  // key within the tile == TMEM lane
-        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        const float sl2 = L.scale_log2;
+        // Warp w: keys 32*(w%4) .. +31 (its TMEM lane quarter), query-row columns
+        // 32*(w/4) .. +31 of every 128-column block; the four column parts of a
+        // key are added at the end.
+        const int quarter = warp & 3, part = warp >> 2;
+        const int j = quarter * 32 + lane;  // key within the tile == TMEM lane
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const float2 sl2v = make_float2(L.scale_log2, L.scale_log2);
         float2 acc[4];  // 8 independent partial sums, in packed pairs
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
@@ -162,42 +173,48 @@ __global__ void __launch_bounds__(192, 1) score_kernel(const __grid_constant__ S
         for (int b = 0; b < NBLK; ++b) {
             const int sb = b % NB;
             const int h = g * L.G + b / n_rb;
-            const int i0 = (b % n_rb) * 128;
+            const int i0 = (b % n_rb) * 128 + part * 32;
             const float *lse2 = P.stats + (static_cast<size_t>(u) * L.Hq + h) * L.q + i0;
-            const int n_rows = min(128, L.q - i0);
+            const int n_rows = min(32, L.q - i0);  // may be <= 0 for the ragged last block
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (b / NB) & 1, ab));
             if (!ok) break;
             tc_fence_after();
-            float x[128];
-            {
-                uint32_t r[128];
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    tmem_ld32(lane_addr + sb * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(r[e]);
-            }
+            uint32_t r[32];
+            tmem_ld32(lane_addr + sb * 128 + part * 32, r);
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_free[sb]);
-            const float2 sl2v = make_float2(sl2, sl2);
+            if (n_rows == 32) {
 #pragma unroll
-            for (int c = 0; c < 128; c += 2) {
-                const float2 nl = make_float2(c < n_rows ? -__ldg(lse2 + c) : -INFINITY,
-                                              c + 1 < n_rows ? -__ldg(lse2 + c + 1) : -INFINITY);
-                const float2 arg = ffma2(make_float2(x[c], x[c + 1]), sl2v, nl);
-                acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(arg.x), ex2(arg.y)));
+                for (int c = 0; c < 32; c += 2) {
+                    const float2 nl = make_float2(-__ldg(lse2 + c), -__ldg(lse2 + c + 1));
+                    const float2 arg = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v, nl);
+                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(arg.x), ex2(arg.y)));
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const float2 nl = make_float2(c < n_rows ? -__ldg(lse2 + c) : -INFINITY,
+                                                  c + 1 < n_rows ? -__ldg(lse2 + c + 1) : -INFINITY);
+                    const float2 arg = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v, nl);
+                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(arg.x), ex2(arg.y)));
+                }
             }
         }
-        if (ok && j < n_valid)
+        float *red = reinterpret_cast<float *>(smem + SM::kOffRed);
+        red[part * 128 + j] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                              ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+        // All score warps leave the loop together (the abort flag is CTA-wide and
+        // every wait is bounded), so this barrier is always reached by all 512.
+        bar_sync(1, kScoreThreads);
+        if (part == 0 && ok && j < n_valid)
             P.scores[static_cast<size_t>(g) * L.C + (key0 - L.a) + j] =
-                ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-                ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+                (red[j] + red[128 + j]) + (red[256 + j] + red[384 + j]);
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kScoreMma) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }

@@ -268,10 +268,10 @@ spava_status run_scores(const Layer &L, const void *q, const void *k, float *sco
     if (blocks == 0) return SPAVA_OK;
     if (L.d == 128) {
         SPAVA_TRY(set_smem(score_kernel<128>, ScoreSmem<128>::kAlloc));
-        score_kernel<128><<<static_cast<unsigned>(blocks), 192, ScoreSmem<128>::kAlloc, st>>>(p);
+        score_kernel<128><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<128>::kAlloc, st>>>(p);
     } else {
         SPAVA_TRY(set_smem(score_kernel<64>, ScoreSmem<64>::kAlloc));
-        score_kernel<64><<<static_cast<unsigned>(blocks), 192, ScoreSmem<64>::kAlloc, st>>>(p);
+        score_kernel<64><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<64>::kAlloc, st>>>(p);
     }
     return launched();
 }
@@ -608,10 +608,10 @@ extern "C" spava_status spava_score_noalloc(const spava_config *cfg, const void 
     if (blocks == 0) return SPAVA_OK;
     if (L.d == 128) {
         SPAVA_TRY(set_smem(score_kernel<128>, ScoreSmem<128>::kAlloc));
-        score_kernel<128><<<static_cast<unsigned>(blocks), 192, ScoreSmem<128>::kAlloc, st>>>(p);
+        score_kernel<128><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<128>::kAlloc, st>>>(p);
     } else {
         SPAVA_TRY(set_smem(score_kernel<64>, ScoreSmem<64>::kAlloc));
-        score_kernel<64><<<static_cast<unsigned>(blocks), 192, ScoreSmem<64>::kAlloc, st>>>(p);
+        score_kernel<64><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<64>::kAlloc, st>>>(p);
     }
     return launched();
 }
