@@ -127,37 +127,61 @@ __global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, con
     }
 }
 
-// Packed passing K/V: row r of KV head g is the anchor row r (r < a) or the
-// s-th kept key of chunk u (r = pcum[u] + s).  One warp per packed row: the
-// first half copies the K row, the second half the V row, 16 bytes per lane.
+// Packed passing K/V: packed row `row` = g*L + r of KV head g is the anchor row r
+// (r < a) or the s-th kept key of chunk u (r = pcum[u] + s).  HBM-bound gather:
+// persistent warps walk groups of 32 packed rows; lane i resolves the source of
+// row i with one coalesced index load, the sources are shuffled out, and rows are
+// copied 8 at a time (first half-warp K, second half V, 16 bytes per lane) with
+// all 8 loads of a lane issued before its stores.
+constexpr int kPackThreads = 256;
+constexpr int kPackBatch = 8;
+
+__device__ __forceinline__ int packed_source(const Layer &L, const int32_t *idx, int g, int r) {
+    if (r < L.a) return r;
+    int u = 0;
+    while (u + 1 < L.n_chunks - 1 && r >= L.pcum[u + 1]) ++u;
+    return idx[(static_cast<size_t>(u) * L.Hkv + g) * L.l + (r - L.pcum[u])];
+}
+
 template <int D>
-__global__ void __launch_bounds__(256) pack_kernel(const Layer L, const __nv_bfloat16 *K,
-                                                   const __nv_bfloat16 *V, const int32_t *idx,
-                                                   __nv_bfloat16 *PK, __nv_bfloat16 *PV) {
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(const Layer L, const __nv_bfloat16 *K,
+                                                            const __nv_bfloat16 *V, const int32_t *idx,
+                                                            __nv_bfloat16 *PK, __nv_bfloat16 *PV) {
     constexpr int kChunks = D * 2 / 16;  // 16-byte pieces per row
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    const long long total = static_cast<long long>(L.Hkv) * L.L;
-    if (warp >= total) return;
-    const int g = static_cast<int>(warp / L.L);
-    const int r = static_cast<int>(warp % L.L);
-    int src;
-    if (r < L.a) {
-        src = r;
-    } else {
-        int u = 0;
-        while (u + 1 < L.n_chunks - 1 && r >= L.pcum[u + 1]) ++u;
-        src = idx[(static_cast<size_t>(u) * L.Hkv + g) * L.l + (r - L.pcum[u])];
-    }
     const int half = lane >> 4, c = lane & 15;
-    if (c >= kChunks) return;
-    __nv_bfloat16 *d = (half ? PV : PK) + (static_cast<size_t>(g) * L.L + r) * D;
-    if (src < 0 || src >= L.N) {  // not a token position: write a zero row, read nothing
-        reinterpret_cast<uint4 *>(d)[c] = make_uint4(0, 0, 0, 0);
-        return;
+    const long long total = static_cast<long long>(L.Hkv) * L.L;
+    const long long n_groups = (total + 31) / 32;
+    const long long stride = static_cast<long long>(gridDim.x) * (kPackThreads / 32);
+    const __nv_bfloat16 *src_base = half ? V : K;
+    __nv_bfloat16 *dst_base = half ? PV : PK;
+    for (long long grp = static_cast<long long>(blockIdx.x) * (kPackThreads / 32) + (threadIdx.x >> 5);
+         grp < n_groups; grp += stride) {
+        // Source element offset of this lane's row, or -1 (past the end, or an
+        // index that is not a token position: written as a zero row).
+        const long long row_l = grp * 32 + lane;
+        long long src_l = -1;
+        if (row_l < total) {
+            const int g = static_cast<int>(row_l / L.L);
+            const int src = packed_source(L, idx, g, static_cast<int>(row_l % L.L));
+            if (src >= 0 && src < L.N) src_l = (static_cast<long long>(src) * L.Hkv + g) * D;
+        }
+#pragma unroll 1
+        for (int b = 0; b < 32; b += kPackBatch) {
+            uint4 v[kPackBatch];
+#pragma unroll
+            for (int k = 0; k < kPackBatch; ++k) {
+                const long long so = __shfl_sync(0xffffffffu, src_l, b + k);
+                v[k] = make_uint4(0, 0, 0, 0);
+                if (so >= 0 && c < kChunks) v[k] = __ldg(reinterpret_cast<const uint4 *>(src_base + so) + c);
+            }
+#pragma unroll
+            for (int k = 0; k < kPackBatch; ++k) {
+                const long long row = grp * 32 + b + k;
+                if (row < total && c < kChunks) reinterpret_cast<uint4 *>(dst_base + row * D)[c] = v[k];
+            }
+        }
     }
-    const __nv_bfloat16 *s = (half ? V : K) + (static_cast<size_t>(src) * L.Hkv + g) * D;
-    reinterpret_cast<uint4 *>(d)[c] = __ldg(reinterpret_cast<const uint4 *>(s) + c);
 }
 
 // Query rows: O = sum_s w_s O_s / sum_s w_s, w_s = 2^(lse2_s - max), over the

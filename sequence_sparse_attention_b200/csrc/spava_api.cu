@@ -285,17 +285,23 @@ spava_status run_topk(const Layer &L, const float *scores, int32_t *idx, cudaStr
 
 spava_status run_pack(const Layer &L, const void *k, const void *v, const int32_t *idx, void *pk,
                       void *pv, cudaStream_t st) {
-    const int64_t warps = static_cast<int64_t>(L.Hkv) * L.L;
-    if (warps == 0) return SPAVA_OK;
-    const int64_t blocks = (warps + 7) / 8;
+    const int64_t rows = static_cast<int64_t>(L.Hkv) * L.L;
+    if (rows == 0) return SPAVA_OK;
+    // Persistent grid: a few blocks per SM, each warp walking 32-row groups.
+    int dev = 0, n_sm = 148;
+    SPAVA_CUDA(cudaGetDevice(&dev));
+    SPAVA_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+    const int64_t groups = (rows + 31) / 32;
+    const int64_t want = (groups + kPackThreads / 32 - 1) / (kPackThreads / 32);
+    const int64_t blocks = std::min<int64_t>(want, static_cast<int64_t>(n_sm) * 8);
     auto K = static_cast<const __nv_bfloat16 *>(k);
     auto V = static_cast<const __nv_bfloat16 *>(v);
     auto PK = static_cast<__nv_bfloat16 *>(pk);
     auto PV = static_cast<__nv_bfloat16 *>(pv);
     if (L.d == 128)
-        pack_kernel<128><<<static_cast<unsigned>(blocks), 256, 0, st>>>(L, K, V, idx, PK, PV);
+        pack_kernel<128><<<static_cast<unsigned>(blocks), kPackThreads, 0, st>>>(L, K, V, idx, PK, PV);
     else
-        pack_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, st>>>(L, K, V, idx, PK, PV);
+        pack_kernel<64><<<static_cast<unsigned>(blocks), kPackThreads, 0, st>>>(L, K, V, idx, PK, PV);
     return launched();
 }
 
