@@ -39,9 +39,13 @@ METRIC = "approx-attn prefill tokens/s per layer on 1 B200; % BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNELS_PER_STEP = 6   # stats, scores, top-l, pack, attention, query merge
 
-# DRAM traffic of one attention launch from an ncu capture (profiles/), valid
-# only while the kernel source is unchanged (sha256 of attn_kernel.cuh).
-PROFILED_TRAFFIC = {"kernel_sha256": None, "bytes_per_launch": None, "source": None}
+# DRAM traffic of one attention launch on the 128K layer, from the single-pass
+# ncu capture summarised in profiles/ (dram__bytes_read.sum + dram__bytes_write.sum);
+# valid only while the sources that decide it are unchanged (KERNEL_FILES).
+PROFILED_TRAFFIC = {"kernel_sha256": "2e4a7c51b02352620939b499384e59d41a1888533ffdb8bc15b0c4737f0fdd7d",
+                    "bytes_per_launch": 2844257024 + 1082235392, "workload": "128k",
+                    "source": "profiles/attn_kernel_128k_launches.md"}
+KERNEL_FILES = ("attn_kernel.cuh", "plan.cuh", "sm100.cuh")
 
 
 def peaks():
@@ -54,9 +58,11 @@ def peaks():
 
 
 def kernel_sha() -> str:
-    p = os.path.join(ROOT, "sequence_sparse_attention_b200", "csrc", "attn_kernel.cuh")
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    h = hashlib.sha256()
+    for name in KERNEL_FILES:
+        with open(os.path.join(ROOT, "sequence_sparse_attention_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 class ClockSampler:
@@ -310,7 +316,7 @@ def run_ours(args, world, rank, local):
     achieved = flops / (per["attn"] / 1e3) / 1e12
     peak = pk_.get("bf16_tflops_sustained") or pk_.get("bf16_tflops")
     traffic = None
-    if PROFILED_TRAFFIC["kernel_sha256"] == kernel_sha():
+    if PROFILED_TRAFFIC["kernel_sha256"] == kernel_sha() and PROFILED_TRAFFIC["workload"] == w.name:
         traffic = PROFILED_TRAFFIC["bytes_per_launch"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,

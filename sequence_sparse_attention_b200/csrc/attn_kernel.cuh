@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layer &L = P.L;
-    const Item it = decode_item(P.groups, P.n_groups, blockIdx.x, L.Hq);
+    const Item it = decode_item(P.groups, P.n_groups, blockIdx.x, L.Hq, L.G);
     Seg segs[kMaxSegs];
     const int ns = build_segments(L, it, segs);
     const int T = count_tiles(segs, ns);

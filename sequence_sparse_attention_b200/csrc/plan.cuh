@@ -44,8 +44,10 @@ struct Layer {
     int32_t pcum[kMaxChunks + 1];      // packed row where P_u starts; pcum[0] = a
 };
 
-// A run of work items of one kind and one chunk/segment; items inside a group
-// are (row tile descending, head ascending) so consecutive CTAs share a KV head.
+// A run of work items of one kind and one chunk/segment.  Items inside a group
+// are ordered (KV head, row tile descending, query head of that KV head): the
+// CTAs resident at any moment then work on one KV head's packed passing K/V and
+// chunks, which fit in L2, and within a KV head the costlier row tiles go first.
 struct Group {
     int32_t kind, sub, n_rt, item_begin;
 };
@@ -62,16 +64,19 @@ __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 __host__ __device__ inline int pair_of(int H, int v) { return v < H ? v : 2 * H - 1 - v; }
 
-__host__ __device__ inline Item decode_item(const Group *groups, int n_groups, int b, int Hq) {
+__host__ __device__ inline Item decode_item(const Group *groups, int n_groups, int b, int Hq,
+                                            int G) {
     int k = 0;
     while (k + 1 < n_groups && b >= groups[k + 1].item_begin) ++k;
     const Group &g = groups[k];
     const int i = b - g.item_begin;
+    const int per_kv = g.n_rt * G;  // items of one KV head
+    const int rem = i % per_kv;
     Item it;
     it.kind = g.kind;
     it.sub = g.sub;
-    it.rt = g.n_rt - 1 - i / Hq;
-    it.h = i % Hq;
+    it.rt = g.n_rt - 1 - rem / G;
+    it.h = (i / per_kv) * G + rem % G;
     return it;
 }
 

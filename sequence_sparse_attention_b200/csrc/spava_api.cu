@@ -91,8 +91,8 @@ int item_tiles(const Layer &L, const Item &it) {
 // Groups of the attention launch, most expensive first: the hardware block
 // scheduler hands out CTAs in index order, so a cost-descending order is a
 // longest-processing-time-first schedule over the SMs.  Inside a group, items
-// run row tile descending (cost descending) with the heads of one KV group
-// adjacent (shared K/V tiles in L2).
+// run KV head by KV head, row tile descending, with the query heads of a KV
+// head adjacent (shared K/V tiles in L2; see decode_item).
 int plan_attention(const Layer &L, bool stats, Group *out) {
     struct G { Group g; int cost; };
     std::vector<G> gs;
