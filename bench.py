@@ -44,7 +44,7 @@ KERNELS_PER_STEP = 6   # stats, scores, top-l, pack, attention, query merge
 # valid only while the sources that decide it are unchanged (KERNEL_FILES).
 PROFILED_TRAFFIC = {"kernel_sha256": "2e4a7c51b02352620939b499384e59d41a1888533ffdb8bc15b0c4737f0fdd7d",
                     "bytes_per_launch": 2844257024 + 1082235392, "workload": "128k",
-                    "source": "profiles/attn_kernel_128k_launches.md"}
+                    "source": "profiles/attn_kernel_128k_dram.md"}
 KERNEL_FILES = ("attn_kernel.cuh", "plan.cuh", "sm100.cuh")
 
 
