@@ -145,12 +145,21 @@ def dist_setup(n_gpus: int):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank value over all ranks (the job is as slow as its slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, steps: int, ms_rank: float, world: int) -> tuple:
+    """Whole-job tokens/s: every rank processes its own layer (weak scaling); the
+    elapsed time is the slowest rank's.  Returns (tokens/s, ms per step)."""
+    ms = max_over_ranks(ms_rank, world)
+    return world * tokens_per_rank * steps / (ms / 1e3), ms / steps
 
 
 def barrier(world: int):
@@ -302,12 +311,10 @@ def run_ours(args, world, rank, local):
     clocks = sampler.summary()
     if sp.device_status():
         raise RuntimeError("kernel status set during the timed region")
-    ms_total = max_over_ranks(start.elapsed_time(end), world)
+    tokens_per_s, ms_step = job_throughput(w.N, args.steps, start.elapsed_time(end), world)
     names = ["score", "topk", "pack", "attn"]
     per = {n: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
            for i, n in enumerate(names)}
-    ms_step = ms_total / args.steps
-    tokens_per_s = world * w.N * args.steps / (ms_total / 1e3)
 
     # ---- roofline of the dominant kernel (approximate attention)
     pk_, pe = peaks()

@@ -145,6 +145,14 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
  * SPAVA_ERR_TIMEOUT if bit 0 was set, SPAVA_OK otherwise. */
 spava_status spava_device_status(void *ws, size_t ws_bytes, void *stream, int32_t *flags);
 
+/* Self-test of the failure path (the pages have no counterpart): launches one
+ * thread that waits on a barrier nothing arrives on.  Its bounded wait gives up
+ * after about two seconds, sets bit 0 of the workspace status word and the
+ * kernel returns, leaving the context usable; spava_device_status() then
+ * reports SPAVA_ERR_TIMEOUT and clears the bit.  Needs the first 256 bytes of a
+ * workspace (256-byte aligned). */
+spava_status spava_selftest_wait_timeout(void *ws, size_t ws_bytes, void *stream);
+
 /* Exact number of (row, key) pairs per query head that spava_attn attends,
  * by row class: pairs[0] anchor rows, pairs[1] context rows, pairs[2] query
  * rows.  Algorithmic FLOPs of spava_attn = 4 * d * Hq * (sum of the three).

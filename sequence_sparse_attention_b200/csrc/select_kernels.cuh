@@ -225,4 +225,23 @@ __global__ void __launch_bounds__(256) merge_kernel(const Layer L, const float *
     if (lane == 0 && lse) lse[static_cast<size_t>(h) * L.N + t] = (m + __log2f(wsum)) * 0.69314718055994531f;
 }
 
+// Failure-path self-test: one thread waits on an mbarrier that nothing ever
+// arrives on.  The bounded wait gives up after kWaitLimitCycles, flags the
+// workspace status word and the kernel returns normally -- the same path every
+// pipeline wait takes when a partner stops making progress.
+__global__ void selftest_wait_kernel(int *status) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const AbortState ab{&abort_flag, status};
+        mbar_wait(&bar, 0, ab);  // never completes: returns false after the limit
+    }
+}
+
 }  // namespace spava

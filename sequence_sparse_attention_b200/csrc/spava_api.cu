@@ -479,6 +479,13 @@ spava_status spava_device_status(void *ws, size_t ws_bytes, void *stream, int32_
     return (h & kStatusTimeout) ? SPAVA_ERR_TIMEOUT : SPAVA_OK;
 }
 
+spava_status spava_selftest_wait_timeout(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws || ws_bytes < 256) return SPAVA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return SPAVA_ERR_MISALIGNED;
+    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<int *>(ws));
+    return launched();
+}
+
 spava_status spava_attended_pairs(const spava_config *cfg, int64_t pairs[3], int64_t *per_host) {
     Layer L;
     SPAVA_TRY(make_layer(cfg, &L));

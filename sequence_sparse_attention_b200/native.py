@@ -20,7 +20,8 @@ STATUS_NAMES = {0: "SPAVA_OK", 1: "SPAVA_ERR_INVALID_ARG", 2: "SPAVA_ERR_UNSUPPO
 EXPORTS = ("spava_workspace_size", "spava_packed_len", "spava_score", "spava_topk_select",
            "spava_pack_passing", "spava_attn", "spava_prefill_attention",
            "spava_prefill_attention_host", "spava_device_status", "spava_attended_pairs",
-           "spava_status_string", "spava_last_cuda_error", "spava_score_noalloc")
+           "spava_status_string", "spava_last_cuda_error", "spava_score_noalloc",
+           "spava_selftest_wait_timeout")
 
 
 class SpavaConfig(ctypes.Structure):
@@ -73,6 +74,7 @@ def load() -> ctypes.CDLL:
         "spava_device_status": [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)],
         "spava_attended_pairs": [cfgp, i64p, i64p],
         "spava_score_noalloc": [cfgp, vp, vp, vp, vp],
+        "spava_selftest_wait_timeout": [vp, sz, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)

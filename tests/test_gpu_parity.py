@@ -29,6 +29,19 @@ CASES = {
                              l=45, frame=64, jitter=0.1, heavy_frac=0.05, seed=15),
     "long_anchor": Workload("long_anchor", H=2, Hq=4, Hkv=4, d=128, N=1800, a=300, q=257, l=160,
                             frame=32, seed=16),
+    # no passing blocks at all: anchor + partner + own chunk only
+    "no_passing": Workload("no_passing", H=3, Hq=6, Hkv=2, d=128, N=1400, a=96, q=70, l=0,
+                           frame=32, seed=17),
+    # no anchor and no passing blocks: zero packed rows
+    "empty_packed": Workload("empty_packed", H=2, Hq=4, Hkv=2, d=64, N=900, a=0, q=40, l=0,
+                             frame=32, seed=18),
+    # chunks shorter than one 128-row tile
+    "short_chunks": Workload("short_chunks", H=4, Hq=4, Hkv=2, d=128, N=600, a=30, q=20, l=20,
+                             frame=16, seed=19),
+    # multi-head (G = 1) and a wide GQA group (G = 16)
+    "mha": Workload("mha", H=2, Hq=3, Hkv=3, d=64, N=1100, a=50, q=60, l=40, frame=32, seed=20),
+    "wide_group": Workload("wide_group", H=2, Hq=16, Hkv=1, d=128, N=1000, a=64, q=130, l=64,
+                           frame=32, seed=21),
 }
 
 _cache = {}
@@ -85,7 +98,7 @@ def test_topk_bit_exact_on_fp32_scores(name):
             np.testing.assert_array_equal(idx[u, g], want, err_msg=f"{name} u={u} g={g}")
 
 
-@pytest.mark.parametrize("name", ["tiny", "g7", "no_anchor", "long_anchor"])
+@pytest.mark.parametrize("name", ["tiny", "g7", "no_anchor", "long_anchor", "short_chunks"])
 def test_pack_exact(name):
     w, Q, K, V, ref, _, _ = setup_case(name)
     sp = Spava(Layout.from_workload(w))
