@@ -79,6 +79,45 @@ def check_selection(w: Workload, scores_oracle: np.ndarray, idx_gpu: np.ndarray,
     return n_exact, n_band
 
 
+def unique_mask(w: Workload, idx_gpu: np.ndarray, idx_ref: np.ndarray, rows, heads) -> np.ndarray:
+    """``[len(rows), len(heads)]``: True where the expected output does not
+    depend on how a tie in the selection was broken.
+
+    Two selections that both pass `check_selection` may differ among keys whose
+    scores tie within fp32 resolution.  A context row of chunk v reads the
+    passing blocks of chunks u < v of its KV group (the anchor and query rows
+    read none), so its output is unique only while the selections of every
+    such (u, g) agree.  The rows where they do not are checked with
+    `check_convex` instead."""
+    off = chunk_offsets(w)
+    G = w.Hq // w.Hkv
+    first_diff = np.full(w.Hkv, 2 * w.H, dtype=np.int64)
+    for g in range(w.Hkv):
+        for u in range(2 * w.H - 1):
+            if not np.array_equal(idx_gpu[u, g], idx_ref[u, g]):
+                first_diff[g] = u
+                break
+    rows = np.asarray(rows, dtype=np.int64)
+    v = np.searchsorted(off, rows, side="right") - 1       # chunk of each context row
+    context = (rows >= w.a) & (rows < w.N - w.q)
+    g_of = np.asarray(heads) // G
+    return ~context[:, None] | (v[:, None] <= first_diff[g_of][None, :])
+
+
+def check_convex(O_gpu: np.ndarray, V: torch.Tensor, heads, G: int, what=""):
+    """Outputs whose key set is one of several valid ones: each is a softmax
+    average of value rows of its KV group, so every coordinate lies within that
+    group's value range (plus bf16 rounding).  ``O_gpu[n, len(heads), d]``."""
+    Vf = V.float()
+    lo = Vf.amin(dim=0).cpu().numpy()        # [Hkv, d]
+    hi = Vf.amax(dim=0).cpu().numpy()
+    g_of = np.asarray(heads) // G
+    slack = 2.0 ** -7 * np.maximum(np.abs(lo), np.abs(hi))
+    assert np.isfinite(O_gpu).all(), f"{what}: non-finite output"
+    assert (O_gpu >= (lo - slack)[g_of][None]).all(), f"{what}: below the value range"
+    assert (O_gpu <= (hi + slack)[g_of][None]).all(), f"{what}: above the value range"
+
+
 def check_outputs(O_gpu: np.ndarray, O_ref: np.ndarray, what=""):
     err = np.abs(O_gpu.astype(np.float64) - O_ref)
     assert np.isfinite(O_gpu).all(), f"{what}: non-finite output"

@@ -11,8 +11,8 @@ import pytest
 import torch
 
 import oracle
-from parity_util import (LSE_ABS, SCORE_REL, check_outputs, check_selection, problem, sample_rows,
-                         to_np)
+from parity_util import (LSE_ABS, SCORE_REL, check_convex, check_outputs, check_selection, problem,
+                         sample_rows, to_np, unique_mask)
 from sequence_sparse_attention_b200.api import Layout, Spava
 from sequence_sparse_attention_b200.synth import WORKLOADS, bf16_bits, chunk_offsets, make_inputs
 
@@ -64,7 +64,13 @@ def test_full_size_layer(name):
     rows = sample_rows(w, per_chunk=8, seed=1)
     O_ref, lse_ref = oracle.prefill_rows(p, Qb, Kb, Vb, idx_ref, rows, heads)
     O_got = to_np(O[torch.from_numpy(rows).cuda()][:, heads])
-    mx, mean = check_outputs(O_got, O_ref, name)
+    # rows that read a passing block whose selection broke an fp32 tie the other
+    # way have several correct outputs: checked for validity only
+    uniq = unique_mask(w, idx_h, idx_ref, rows, heads)
+    assert uniq.mean() > 0.5
+    mx, mean = check_outputs(O_got[uniq], O_ref[uniq], name)
+    check_convex(O_got[~uniq], V, heads, G, name)
     lse_got = to_np(lse[heads][:, torch.from_numpy(rows).cuda()]).T
-    np.testing.assert_allclose(lse_got, lse_ref, atol=LSE_ABS, rtol=0)
-    print(f"{name}: selections exact {n_exact}, in-band {n_band}; O max {mx:.2e} mean {mean:.2e}")
+    np.testing.assert_allclose(lse_got[uniq], lse_ref[uniq], atol=LSE_ABS, rtol=0)
+    print(f"{name}: selections exact {n_exact}, in-band {n_band}; O max {mx:.2e} mean {mean:.2e};"
+          f" tie-dependent outputs {int((~uniq).sum())}")

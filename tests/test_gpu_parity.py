@@ -8,7 +8,8 @@ import pytest
 import torch
 
 import oracle
-from parity_util import (LSE_ABS, SCORE_REL, OracleRun, check_outputs, check_selection, to_np)
+from parity_util import (LSE_ABS, SCORE_REL, OracleRun, check_convex, check_outputs, check_selection,
+                         to_np, unique_mask)
 from sequence_sparse_attention_b200.api import Layout, Spava
 from sequence_sparse_attention_b200.synth import WORKLOADS, Workload, chunk_offsets, make_inputs
 
@@ -137,9 +138,17 @@ def test_prefill_end_to_end(name):
     sp = Spava(Layout.from_workload(w))
     O, lse, idx = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda(), want_idx=True)
     device_clean(sp)
-    check_selection(w, ref.scores, idx.cpu().numpy(), range(w.Hkv))
-    check_outputs(to_np(O), O_ref, name)
-    np.testing.assert_allclose(to_np(lse).T, lse_ref, atol=LSE_ABS, rtol=0)
+    idx_h = idx.cpu().numpy()
+    check_selection(w, ref.scores, idx_h, range(w.Hkv))
+    # Where the fp32 scores broke a tie the other way than the fp64 oracle, the
+    # rows reading that passing block have several correct outputs.
+    heads = list(range(w.Hq))
+    uniq = unique_mask(w, idx_h, ref.idx, np.arange(w.N), heads)
+    assert uniq.mean() > 0.5
+    O_np = to_np(O)
+    check_outputs(O_np[uniq], O_ref[uniq], name)
+    check_convex(O_np[~uniq], V, heads, w.Hq // w.Hkv, name)
+    np.testing.assert_allclose(to_np(lse).T[uniq], lse_ref[uniq], atol=LSE_ABS, rtol=0)
 
 
 def test_values_one_give_ones():
