@@ -1,27 +1,34 @@
-// attn_kernel.cuh -- approximate attention with online softmax on tcgen05/TMEM.
+// attn_kernel.cuh -- approximate attention, two query tiles per CTA, the
+// tensor core working on one tile while the other tile's softmax runs.
 //
 // "Riepilogo Tecnico: APB-V", Metodologia, "Meccanismo di Attenzione
 // Approssimata" / "Computazione": every row attends its key segments (anchor,
 // passing blocks, partner chunk, own chunk; plan.cuh); "Forward Fuso di
 // Contesto e Query": query rows are computed as per-segment partials carrying
-// their log-sum-exp, merged later.  The same kernel in STATS mode computes the
-// per-chunk softmax statistics of the query block that the scoring pass needs.
+// their log-sum-exp, merged later.
 //
-// One CTA = one work item = 128 query rows of one head.  Warp roles:
-//   warps 0-7  softmax: two warps per TMEM lane quarter, each taking one half
-//              of the 128 keys of a tile; online softmax with conditional
-//              rescaling (the running max only moves when it grows by more than
-//              2^8), P written back into TMEM as bf16
-//   warp  8    TMA producer: Q tile once, then K (and V) tiles through rings
-//   warp  9    MMA issuer: S = Q K^T (SS, K-major/K-major) into one of two S
-//              buffers in TMEM; O += P V (P from TMEM, V MN-major in smem)
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D), P0 [384,448),
-// P1 [448,512) (bf16 pairs).  P has its own columns, so S_{j+2} is issued right
-// behind PV_j without waiting for PV_j to finish; the softmax writes P_{j+2} over
-// P_j only after S_{j+2} has completed, and that completion (tcgen05.commit
-// tracks every earlier MMA of the issuing thread) implies PV_j has completed.
-// MMAs with different accumulators are not ordered by the hardware, so every
-// hand-off goes through an mbarrier.
+// One CTA = two adjacent 128-row tiles A (x = 0) and B (x = 1) of one head; B
+// may be absent at the end of a region.  Both see the same key sequence, except
+// that B sees one more tile (its own diagonal) when the sequence ends in a
+// causal segment.  Warp roles:
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: warp w owns the
+//              TMEM lane quarter w % 4, i.e. 32 rows, and all 128 keys of every
+//              key tile -- no exchange between warps.  Online softmax with
+//              conditional rescaling (the running max only moves when it grows
+//              by more than 2^8), P written back into TMEM as bf16.
+//   warp  8    TMA producer: Q_A, Q_B once, then K (one tile ahead) and V rings
+//   warp  9    MMA issuer, per key tile j:
+//                PV_A(j)  S_A(j+1)  PV_B(j)  S_B(j+1)
+//              so S_X(j+1) enters the tensor pipe right behind PV_X(j) while the
+//              other tile's softmax is running.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
+// P_X(j) (bf16 pairs) goes to S_X's columns [0,64) once the softmax holds all of
+// S_X(j) in registers.  The tcgen05.mma operations of one thread run in issue
+// order, so S_X(j+1), issued right behind PV_X(j), overwrites P_X(j) only after
+// PV_X(j) has read it (the order the CUTLASS Blackwell FMHA also relies on).
+// The commit that announces S_X(j+1) tracks every earlier MMA of the thread,
+// PV_X(j) included, so whenever the softmax of tile X sees a new S, O_X is
+// stable and can be rescaled without a further wait.
 #pragma once
 
 #include "plan.cuh"
@@ -42,42 +49,73 @@ struct AttnParams {
     int *status;        // workspace status word
 };
 
-template <int D, bool STATS>
+// sm_100 allows at most 227 KiB of dynamic shared memory per CTA.
+constexpr int kMaxDynSmem = 232448;
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
 struct AttnSmem {
     static constexpr int kPanels = D / 64;
     static constexpr int kTile = kRowTile * D * 2;  // one 128-row bf16 tile
-    static constexpr int KS = STATS ? 4 : 3;
-    static constexpr int VS = STATS ? 1 : (D == 128 ? 2 : 3);  // STATS mode leaves V unused
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kTile;
+    // Each K tile feeds two S MMAs and each V tile two PVs, so the rings turn
+    // over half as often per MMA as with one query tile.
+    static constexpr int KS = D == 128 ? 2 : 4;
+    static constexpr int VS = D == 128 ? 2 : 3;
+    static constexpr int kOffQ = 0;  // Q_A, Q_B
+    static constexpr int kOffK = 2 * kTile;
     static constexpr int kOffV = kOffK + KS * kTile;
-    static constexpr int kOffBar = kOffV + (STATS ? 0 : VS) * kTile;
-    static constexpr int kNumBar = 1 + 2 * KS + 2 * VS + 8 + 1;
-    static constexpr int kOffRed = kOffBar + kNumBar * 8;        // row-max / row-sum exchange
-    static constexpr int kOffMisc = kOffRed + 6 * kRowTile * 4;
+    static constexpr int kOffBar = kOffV + VS * kTile;
+    static constexpr int kNumBar = 1 + 2 * KS + 2 * VS + 6 + 1;
+    static constexpr int kOffMisc = kOffBar + kNumBar * 8;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
 };
+static_assert(AttnSmem<128>::kAlloc <= kMaxDynSmem, "attention smem over budget");
+static_assert(AttnSmem<64>::kAlloc <= kMaxDynSmem, "attention smem over budget");
 
-// sm_100 allows at most 227 KiB of dynamic shared memory per CTA.
-constexpr int kMaxDynSmem = 232448;
-static_assert(AttnSmem<128, false>::kAlloc <= kMaxDynSmem, "attention smem over budget");
-static_assert(AttnSmem<128, true>::kAlloc <= kMaxDynSmem, "statistics smem over budget");
-static_assert(AttnSmem<64, false>::kAlloc <= kMaxDynSmem, "attention smem over budget");
+constexpr int kSoftWarps = 8;  // 4 per query tile
+constexpr int kAttnThreads = (kSoftWarps + 2) * 32;
+constexpr int kProducerWarp = kSoftWarps;
+constexpr int kMmaWarp = kSoftWarps + 1;
+constexpr int kColO = 256;  // O_A; O_B at kColO + 128
 
-constexpr int kSoftmaxWarps = 8;
-constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-constexpr int kProducerWarp = kSoftmaxWarps;
-constexpr int kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kAttnThreads = (kSoftmaxWarps + 2) * 32;
-constexpr int kHalf = kKeyTile / 2;  // keys of a tile handled by one softmax warp
-constexpr uint32_t kTmemCols = 512;
-constexpr int kColO = 256;
-constexpr int kColP = 384;
+// Work item = row tiles 2p and 2p+1 of a region.  Inside a group: KV head by KV
+// head, pairs in descending cost, the query heads of a KV head adjacent.
+__host__ __device__ inline int pair_count(int n_rt) { return (n_rt + 1) / 2; }
 
-template <int D, bool STATS>
+__host__ __device__ inline Item decode_pair_item(const Group *groups, int n_groups, int b, int G) {
+    int k = 0;
+    while (k + 1 < n_groups && b >= groups[k + 1].item_begin) ++k;
+    const Group &g = groups[k];
+    const int i = b - g.item_begin;
+    const int np = pair_count(g.n_rt);
+    const int per_kv = np * G;
+    const int rem = i % per_kv;
+    Item it;
+    it.kind = g.kind;
+    it.sub = g.sub;
+    it.rt = 2 * (np - 1 - rem / G);  // first row tile of the pair
+    it.h = (i / per_kv) * G + rem % G;
+    return it;
+}
+
+// Max of 128 values: four independent chains of 3-input max.
+__device__ __forceinline__ float max128(const float (&x)[128]) {
+    float m[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = fmax3(x[k], x[4 + k], x[8 + k]);
+#pragma unroll
+    for (int c = 12; c + 8 <= 124; c += 8)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m[k] = fmax3(m[k], x[c + k], x[c + 4 + k]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], x[124 + k]);
+    return fmaxf(fmax3(m[0], m[1], m[2]), m[3]);
+}
+
+template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
-    using SM = AttnSmem<D, STATS>;
+    using SM = AttnSmem<D>;
     constexpr int KS = SM::KS, VS = SM::VS;
     constexpr uint32_t kIdescS = idesc_bf16_f32(128, kKeyTile, 0, 0);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
@@ -91,22 +129,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     uint64_t *k_empty = k_full + KS;
     uint64_t *v_full = k_empty + KS;
     uint64_t *v_empty = v_full + VS;
-    uint64_t *s_full = v_empty + VS;
-    uint64_t *s_free = s_full + 2;
-    uint64_t *p_full = s_free + 2;
-    uint64_t *pv_done = p_full + 2;
-    uint64_t *mma_drain = pv_done + 2;
+    uint64_t *s_full = v_empty + VS;  // [2]: S_X(j) in TMEM
+    uint64_t *p_full = s_full + 2;    // [2]: P_X(j) in TMEM
+    uint64_t *o_done = p_full + 2;    // [2]: the last PV_X has completed
+    uint64_t *mma_drain = o_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layer &L = P.L;
-    const Item it = decode_item(P.groups, P.n_groups, blockIdx.x, L.Hq, L.G);
+    const Item it = decode_pair_item(P.groups, P.n_groups, blockIdx.x, L.G);
+    Item it_b = it;
+    it_b.rt = it.rt + 1;
+    int r0A, eA, r0B, eB;
+    item_rows(L, it, r0A, eA);
+    item_rows(L, it_b, r0B, eB);
+    const bool hasB = eB > r0B;
     Seg segs[kMaxSegs];
-    const int ns = build_segments(L, it, segs);
+    const int ns = build_segments(L, hasB ? it_b : it, segs);
     const int T = count_tiles(segs, ns);
-    int row0, row_end;
-    item_rows(L, it, row0, row_end);
+    // A causal last segment starts on a tile boundary of the region, so its last
+    // tile for B is B's diagonal, which lies beyond every row of A.
+    const int TA = (hasB && ns > 0 && segs[ns - 1].causal) ? T - 1 : T;
+    const int TB = hasB ? T : 0;
     const int g = it.h / L.G;
 
     if (threadIdx.x == 0) {
@@ -121,9 +166,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], kSoftmaxThreads);
-            mbar_init(&p_full[i], kSoftmaxThreads);
-            mbar_init(&pv_done[i], 1);
+            mbar_init(&p_full[i], 128);
+            mbar_init(&o_done[i], 1);
         }
         mbar_init(mma_drain, 1);
         *abort_flag = 0;
@@ -132,11 +176,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     if (warp == kProducerWarp && lane == 0) {
         tma_prefetch(&P.tmQ);
         tma_prefetch(&P.tmK);
-        if (!STATS) {
-            tma_prefetch(&P.tmV);
-            tma_prefetch(&P.tmPK);
-            tma_prefetch(&P.tmPV);
-        }
+        tma_prefetch(&P.tmV);
+        tma_prefetch(&P.tmPK);
+        tma_prefetch(&P.tmPV);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -148,15 +190,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_expect_tx(q_full, SM::kTile);
+            mbar_expect_tx(q_full, hasB ? 2 * SM::kTile : SM::kTile);
             for (int p = 0; p < SM::kPanels; ++p)
-                tma_load_3d(smem + SM::kOffQ + p * 16384, &P.tmQ, p * 64, it.h, row0, q_full);
+                tma_load_3d(smem + SM::kOffQ + p * 16384, &P.tmQ, p * 64, it.h, r0A, q_full);
+            if (hasB)
+                for (int p = 0; p < SM::kPanels; ++p)
+                    tma_load_3d(smem + SM::kOffQ + SM::kTile + p * 16384, &P.tmQ, p * 64, it.h, r0B,
+                                q_full);
             int k_last[KS], v_last[VS];
             for (int i = 0; i < KS; ++i) k_last[i] = -1;
             for (int i = 0; i < VS; ++i) v_last[i] = -1;
-            // K runs one tile ahead of V: S_{j+1} needs K_{j+1} before PV_j needs V_j.
+            // K runs one tile ahead of V: S_X(j+1) needs K_{j+1} right behind PV_X(j).
             TileCursor kc, vc;
-            bool live = true;
             auto load_k = [&](int j) -> bool {
                 const int ks = j % KS;
                 if (j >= KS && !mbar_wait(&k_empty[ks], ((j / KS) - 1) & 1, ab)) return false;
@@ -191,10 +236,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 vc.advance(segs);
                 return true;
             };
-            if (T > 0) live = load_k(0);
+            bool live = T > 0 ? load_k(0) : true;
             for (int j = 0; live && j < T; ++j) {
                 if (j + 1 < T) live = load_k(j + 1);
-                if (live && !STATS) live = load_v(j);
+                if (live) live = load_v(j);
             }
             // Every load this thread issued has landed before the CTA may exit.
             mbar_wait_drain(q_full, 0);
@@ -206,61 +251,76 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            // Descriptors are built once; a K-step or a ring stage only adds its
-            // byte offset / 16 to the start-address field (addresses < 256 KiB, so
-            // the 14-bit field never carries into the next one).  This keeps the
-            // issuing thread down to a couple of instructions per MMA.
-            constexpr int NK = D / 16;  // K-steps of S = Q K^T
-            uint64_t qd[NK];            // A descriptors of the Q tile, one per K-step
-            const uint64_t q_desc = sdesc_sw128(smem_u32(smem + SM::kOffQ), 16, 1024);
+            // Descriptors built once; a K-step or a ring stage adds its byte
+            // offset / 16 to the start-address field.
+            constexpr int NK = D / 16;
+            uint64_t qd[2][NK];
             const uint64_t k_desc = sdesc_sw128(smem_u32(smem + SM::kOffK), 16, 1024);
             const uint64_t v_desc = sdesc_sw128(smem_u32(smem + SM::kOffV), 16384, 1024);
 #pragma unroll
-            for (int kk = 0; kk < NK; ++kk) qd[kk] = q_desc + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-            bool ok = mbar_wait(q_full, 0, ab);
-            tc_fence_after();
-            auto issue_s = [&](int j) -> bool {
-                const int ks = j % KS;
-                if (!mbar_wait(&k_full[ks], (j / KS) & 1, ab)) return false;
-                tc_fence_after();
-                const uint32_t d_s = tmem + (j & 1) * kKeyTile;
-                const uint64_t kd = k_desc + static_cast<uint64_t>((ks * SM::kTile) >> 4);
+            for (int x = 0; x < 2; ++x) {
+                const uint64_t q_desc = sdesc_sw128(smem_u32(smem + SM::kOffQ + x * SM::kTile), 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < NK; ++kk)
+                    qd[x][kk] = q_desc + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            }
+            // S_X(j) = Q_X K_j^T into TMEM columns [128x, 128x+128).
+            auto mma_s = [&](int x, int j) {
+                const uint64_t kd = k_desc + static_cast<uint64_t>(((j % KS) * SM::kTile) >> 4);
+                const uint32_t d_s = tmem + x * kKeyTile;
 #pragma unroll
                 for (int g4 = 0; g4 < NK / 4; ++g4) {
                     const uint64_t kb = kd + static_cast<uint64_t>(g4 * (16384 >> 4));
-                    mma_ss_x4(d_s, qd[4 * g4], qd[4 * g4 + 1], qd[4 * g4 + 2], qd[4 * g4 + 3], kb,
-                              kb + 2, kb + 4, kb + 6, kIdescS, g4 > 0);
+                    mma_ss_x4(d_s, qd[x][4 * g4], qd[x][4 * g4 + 1], qd[x][4 * g4 + 2],
+                              qd[x][4 * g4 + 3], kb, kb + 2, kb + 4, kb + 6, kIdescS, g4 > 0);
                 }
-                tc_commit(&k_empty[ks]);
-                tc_commit(&s_full[j & 1]);
-                return true;
+                tc_commit(&s_full[x]);
             };
-            if (ok) ok = issue_s(0);
-            if (ok && T > 1) ok = issue_s(1);
+            // O_X += P_X(j) V_j.  K-step kb covers keys 16kb..16kb+15: P columns
+            // +8kb inside S_X, V rows +2048 B.
+            auto mma_pv = [&](int x, int j) {
+                const uint32_t a_p = tmem + x * kKeyTile;
+                const uint64_t vd = v_desc + static_cast<uint64_t>(((j % VS) * SM::kTile) >> 4);
+                const uint32_t d_o = tmem + kColO + x * 128;
+                mma_ts_x4(d_o, a_p, a_p + 8, a_p + 16, a_p + 24, vd, vd + 128, vd + 256, vd + 384,
+                          kIdescPV, j > 0);
+                mma_ts_x4(d_o, a_p + 32, a_p + 40, a_p + 48, a_p + 56, vd + 512, vd + 640, vd + 768,
+                          vd + 896, kIdescPV, 1u);
+            };
+            bool ok = mbar_wait(q_full, 0, ab) && (T == 0 || mbar_wait(&k_full[0], 0, ab));
+            tc_fence_after();
+            if (ok && T > 0) {
+                if (TA > 0) mma_s(0, 0);
+                if (TB > 0) mma_s(1, 0);
+                tc_commit(&k_empty[0]);
+            }
             for (int j = 0; ok && j < T; ++j) {
-                if (!STATS) {
-                    if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, ab)) break;
-                    tc_fence_after();
-                    const int vs = j % VS;
-                    if (!mbar_wait(&v_full[vs], (j / VS) & 1, ab)) break;
-                    tc_fence_after();
-                    const uint32_t a_p = tmem + kColP + (j & 1) * (kKeyTile / 2);
-                    const uint64_t vd = v_desc + static_cast<uint64_t>((vs * SM::kTile) >> 4);
-                    // K-step kb covers keys 16kb..16kb+15: P columns +8kb, V rows +2048 B.
-                    mma_ts_x4(tmem + kColO, a_p, a_p + 8, a_p + 16, a_p + 24, vd, vd + 128, vd + 256,
-                              vd + 384, kIdescPV, j > 0);
-                    mma_ts_x4(tmem + kColO, a_p + 32, a_p + 40, a_p + 48, a_p + 56, vd + 512, vd + 640,
-                              vd + 768, vd + 896, kIdescPV, 1u);
-                    tc_commit(&v_empty[vs]);
-                    tc_commit(&pv_done[j & 1]);
+                const int vs = j % VS, kn = j + 1, ks = kn % KS;
+                if (!mbar_wait(&v_full[vs], (j / VS) & 1, ab)) break;
+                bool k_seen = false;
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const int TX = x ? TB : TA;
+                    if (ok && j < TX) {
+                        ok = mbar_wait(&p_full[x], j & 1, ab);
+                        if (!ok) break;
+                        tc_fence_after();
+                        mma_pv(x, j);
+                        if (j + 1 == TX) tc_commit(&o_done[x]);
+                        if (kn < TX) {
+                            if (!k_seen) {
+                                ok = mbar_wait(&k_full[ks], (kn / KS) & 1, ab);
+                                if (!ok) break;
+                                tc_fence_after();
+                                k_seen = true;
+                            }
+                            mma_s(x, kn);
+                        }
+                    }
                 }
-                if (j + 2 < T) {
-                    // S buffer (j&1) is reused by S_{j+2}: the softmax has loaded S_j
-                    // (s_free_j; in attention mode also implied by p_full_j above).
-                    if (!mbar_wait(&s_free[j & 1], (j >> 1) & 1, ab)) break;
-                    tc_fence_after();
-                    if (!issue_s(j + 2)) break;
-                }
+                if (!ok) break;
+                tc_commit(&v_empty[vs]);
+                if (k_seen) tc_commit(&k_empty[ks]);
             }
             // No MMA may still be running when TMEM is released.
             tc_commit(mma_drain);
@@ -269,58 +329,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
-        // Warps 0-7: warp w owns rows 32*(w%4) .. +31 (its TMEM lane quarter) and
-        // the key half kh = w/4 of every tile (keys 64*kh .. +63).  The two warps
-        // of a quarter exchange their partial row maxima through shared memory;
-        // every abort decision is taken jointly with bar.red.and so that both
-        // always reach the same named barriers.
-        const int quarter = warp & 3, kh = warp >> 2;
+        const int x = warp >> 2, quarter = warp & 3;
+        const int TX = x ? TB : TA;
+        const int row0 = x ? r0B : r0A, row_end = x ? eB : eA;
         const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
         const int t = row0 + r;
-        const int pair_bar = 1 + quarter;   // named barrier of the two warps of a quarter
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-        float *red = reinterpret_cast<float *>(smem + SM::kOffRed);  // [2][2][128]
+        const uint32_t col_s = x * kKeyTile, col_o = kColO + x * 128;
         const float sl2 = L.scale_log2;
+        const float2 sl2v = make_float2(sl2, sl2);
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        int sg = 0, kt = 0;
-        for (int j = 0; j < T; ++j) {
-            const Seg &s = segs[sg];
-            const int key0 = s.begin + kt * kKeyTile + kh * kHalf;
+        TileCursor cur;
+        for (int j = 0; j < TX; ++j) {
+            const Seg &s = segs[cur.seg];
+            const int key0 = s.begin + cur.tile * kKeyTile;
             int lim_end = s.end;
             if (s.causal && t + 1 < lim_end) lim_end = t + 1;
-            const int lim = lim_end - key0;  // keys [0, lim) of this half-tile are valid for row r
+            const int lim = lim_end - key0;  // keys [0, lim) of this tile are valid for row r
+            cur.advance(segs);
 
-            const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, ab));
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, ab));
+            if (!ok) break;
             tc_fence_after();
-            float x[kHalf];
+            float xs[kKeyTile];
             {
-                uint32_t u[kHalf];
+                uint32_t u[4][32];
 #pragma unroll
-                for (int c = 0; c < kHalf / 32; ++c)
-                    tmem_ld32(lane_addr + (j & 1) * kKeyTile + kh * kHalf + c * 32,
-                              *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
+                for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + col_s + c * 32, u[c]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < kHalf; ++e) x[e] = __uint_as_float(u[e]);
-            }
-            tc_fence_before();
-            mbar_arrive(&s_free[j & 1]);
-            // P_j overwrites the columns of P_{j-2}; S_j was issued after PV_{j-2},
-            // so S_j's completion (seen above) implies PV_{j-2} has completed.
-            const bool landed = true;
-            if (lim < kHalf) {
+                for (int c = 0; c < 4; ++c) {
+                    reg_fence(u[c]);
 #pragma unroll
-                for (int c = 0; c < kHalf; ++c)
-                    if (c >= lim) x[c] = -INFINITY;
+                    for (int e = 0; e < 32; ++e) xs[c * 32 + e] = __uint_as_float(u[c][e]);
+                }
             }
-            // Partial row max (3-input max, 4 chains), then the pair's exchange.
-            static_assert(kHalf == 64, "max64 covers one half tile");
-            const float mx_mine = max64(x);
-            red[((j & 1) * 2 + kh) * kRowTile + r] = mx_mine;
-            ok = bar_red_and(pair_bar, 64, got && landed);
-            if (!ok) break;
-            const float mx = fmaxf(mx_mine, red[((j & 1) * 2 + (kh ^ 1)) * kRowTile + r]) * sl2;
+            if (lim < kKeyTile) {  // only tiles crossing a segment end or the diagonal
+#pragma unroll
+                for (int c = 0; c < kKeyTile; ++c)
+                    if (c >= lim) xs[c] = -INFINITY;
+            }
+            const float mx = max128(xs) * sl2;
             const float m_new = fmaxf(m_run, mx);
             const bool need = m_new > m_run + 8.0f;
             float alpha = 1.f;
@@ -329,21 +379,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 l_run *= alpha;
                 m_run = m_new;
             }
-            if (!STATS && j > 0 && __any_sync(0xffffffffu, need)) {
-                // O holds the sum up to tile j-1 scaled by the old max: rescale this
-                // warp's half of the O columns once PV_{j-1} has landed.  Both warps
-                // of the quarter see the same rows' `need`, so both come here.
-                const bool landed = __all_sync(
-                    0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, ab));
-                ok = bar_red_and(pair_bar, 64, landed);
-                if (!ok) break;
-                tc_fence_after();
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                // O_X holds the sum up to tile j-1 scaled by the old max, and is
+                // stable: PV_X(j-1) completed before S_X(j) was announced.
 #pragma unroll 1
-                for (int c = 0; c < D / 64; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t u[32];
-                    const uint32_t a = lane_addr + kColO + kh * (D / 2) + c * 32;
+                    const uint32_t a = lane_addr + col_o + c * 32;
                     tmem_ld32(a, u);
                     tmem_wait_ld();
+                    reg_fence(u);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
                     tmem_st32(a, u);
@@ -351,85 +396,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 tmem_wait_st();
             }
             const float mu = (m_run == -INFINITY) ? 0.f : m_run;
-            // Probabilities: exponent arguments and partial sums in packed pairs.
-            const float2 sl2v = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
-            float2 ps[4];
+            const float2 nmu = make_float2(-mu, -mu);
+            float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            // P, 32 keys (16 bf16-pair columns) at a time, over S columns this
+            // warp has already read.
 #pragma unroll
-            for (int k = 0; k < 4; ++k) ps[k] = make_float2(0.f, 0.f);
-            uint32_t u[32];
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const float2 arg = ffma2(make_float2(x[2 * e], x[2 * e + 1]), sl2v, nmu);
-                const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
-                ps[e & 3] = fadd2(ps[e & 3], p);
-                if (!STATS) u[e] = pack_bf16x2(p.x, p.y);
+                for (int e = 0; e < 16; ++e) {
+                    const float2 arg = ffma2(make_float2(xs[c * 32 + 2 * e], xs[c * 32 + 2 * e + 1]), sl2v, nmu);
+                    const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
+                    ps[e & 1] = fadd2(ps[e & 1], p);
+                    pk[e] = pack_bf16x2(p.x, p.y);
+                }
+                tmem_st16(lane_addr + col_s + c * 16, pk);
             }
-            if (STATS) {
-                (void)u;
-            } else {
-                tmem_st32(lane_addr + kColP + (j & 1) * (kKeyTile / 2) + kh * 32, u);
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&p_full[j & 1]);
-            }
-            const float2 pss = fadd2(fadd2(ps[0], ps[1]), fadd2(ps[2], ps[3]));
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&p_full[x]);
+            const float2 pss = fadd2(ps[0], ps[1]);
             l_run += pss.x + pss.y;
-            if (s.begin + (kt + 1) * kKeyTile >= s.end) {
-                ++sg;
-                kt = 0;
-            } else {
-                ++kt;
-            }
         }
 
         // ------------------------------------------------------------ epilogue
-        // Row sum = the two halves' partial sums (same running max in both).
-        float *lred = red + 4 * kRowTile;  // [2][128]
-        lred[kh * kRowTile + r] = l_run;
-        bar_sync(pair_bar, 64);
-        const float l_tot = l_run + lred[(kh ^ 1) * kRowTile + r];
-        const bool valid = ok && t < row_end;
-        const float lse2 = (l_tot > 0.f) ? m_run + __log2f(l_tot) : -INFINITY;
-        if (STATS) {
-            if (valid && kh == 0) {
-                const int i = t - (L.N - L.q);
-                P.stats[(static_cast<size_t>(it.sub) * L.Hq + it.h) * L.q + i] = lse2;
-            }
-        } else if (ok && T > 0) {
-            const bool landed = __all_sync(
-                0xffffffffu, mbar_wait(&pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, ab));
-            if (bar_red_and(pair_bar, 64, landed)) {
+        if (ok && TX > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&o_done[x], 0, ab));
+            if (ok) {
                 tc_fence_after();
-                const float inv = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
-                const int c0 = kh * (D / 2);  // this warp's half of the O columns
+                const bool valid = t < row_end;
+                const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+                const float lse2 = (l_run > 0.f) ? m_run + __log2f(l_run) : -INFINITY;
                 if (it.kind == kQueryPart) {
                     const int i = t - (L.N - L.q);
-                    float *dst = P.part_O + ((static_cast<size_t>(it.sub) * L.Hq + it.h) * L.q + i) * D + c0;
-#pragma unroll
-                    for (int c = 0; c < D / 64; ++c) {
+                    float *dst = P.part_O + ((static_cast<size_t>(it.sub) * L.Hq + it.h) * L.q + i) * D;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
                         uint32_t u[32];
-                        tmem_ld32(lane_addr + kColO + c0 + c * 32, u);
+                        tmem_ld32(lane_addr + col_o + c * 32, u);
                         tmem_wait_ld();
+                        reg_fence(u);
                         if (valid) {
 #pragma unroll
-                            for (int e = 0; e < 32; e += 4) {
-                                float4 f = make_float4(__uint_as_float(u[e]) * inv,
-                                                       __uint_as_float(u[e + 1]) * inv,
-                                                       __uint_as_float(u[e + 2]) * inv,
-                                                       __uint_as_float(u[e + 3]) * inv);
-                                *reinterpret_cast<float4 *>(dst + c * 32 + e) = f;
-                            }
+                            for (int e = 0; e < 32; e += 4)
+                                *reinterpret_cast<float4 *>(dst + c * 32 + e) =
+                                    make_float4(__uint_as_float(u[e]) * inv, __uint_as_float(u[e + 1]) * inv,
+                                                __uint_as_float(u[e + 2]) * inv, __uint_as_float(u[e + 3]) * inv);
                         }
                     }
-                    if (valid && kh == 0)
-                        P.part_lse[(static_cast<size_t>(it.sub) * L.Hq + it.h) * L.q + i] = lse2;
+                    if (valid) P.part_lse[(static_cast<size_t>(it.sub) * L.Hq + it.h) * L.q + i] = lse2;
                 } else {
-                    __nv_bfloat16 *dst = P.O + (static_cast<size_t>(t) * L.Hq + it.h) * D + c0;
-#pragma unroll
-                    for (int c = 0; c < D / 64; ++c) {
+                    __nv_bfloat16 *dst = P.O + (static_cast<size_t>(t) * L.Hq + it.h) * D;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
                         uint32_t u[32];
-                        tmem_ld32(lane_addr + kColO + c0 + c * 32, u);
+                        tmem_ld32(lane_addr + col_o + c * 32, u);
                         tmem_wait_ld();
+                        reg_fence(u);
                         if (valid) {
 #pragma unroll
                             for (int e = 0; e < 32; e += 8) {
@@ -442,8 +465,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                             }
                         }
                     }
-                    if (valid && kh == 0 && P.lse)
-                        P.lse[static_cast<size_t>(it.h) * L.N + t] = lse2 * 0.69314718055994531f;
+                    if (valid && P.lse) P.lse[static_cast<size_t>(it.h) * L.N + t] = lse2 * 0.69314718055994531f;
                 }
             }
         }

@@ -12,6 +12,7 @@
 
 #include "../../include/spava.h"
 #include "attn_kernel.cuh"
+#include "stats_kernel.cuh"
 #include "plan.cuh"
 #include "score_kernel.cuh"
 #include "select_kernels.cuh"
@@ -110,17 +111,20 @@ int plan_attention(const Layer &L, bool stats, Group *out) {
         for (int s = (L.a > 0 ? 0 : 1); s < L.n_chunks + 2; ++s) push(kQueryPart, s, n_qrt);
     }
     std::stable_sort(gs.begin(), gs.end(), [](const G &x, const G &y) { return x.cost > y.cost; });
+    // The statistics pass runs one row tile per CTA, the attention two.
     int begin = 0, n = 0;
     for (auto &g : gs) {
         g.g.item_begin = begin;
-        begin += g.g.n_rt * L.Hq;
+        begin += (stats ? g.g.n_rt : pair_count(g.g.n_rt)) * L.Hq;
         out[n++] = g.g;
     }
     return n;
 }
 
-int64_t plan_items(const Group *g, int n, int Hq) {
-    return n ? static_cast<int64_t>(g[n - 1].item_begin) + static_cast<int64_t>(g[n - 1].n_rt) * Hq : 0;
+int64_t plan_items(const Group *g, int n, int Hq, bool stats) {
+    if (!n) return 0;
+    const int per = stats ? g[n - 1].n_rt : pair_count(g[n - 1].n_rt);
+    return static_cast<int64_t>(g[n - 1].item_begin) + static_cast<int64_t>(per) * Hq;
 }
 
 // ---------------------------------------------------------------- workspace
@@ -225,12 +229,18 @@ spava_status launched() {
 // ---------------------------------------------------------------- launches
 template <int D, bool STATS>
 spava_status launch_attn(AttnParams &p, cudaStream_t st) {
-    using SM = AttnSmem<D, STATS>;
-    const int64_t items = plan_items(p.groups, p.n_groups, p.L.Hq);
+    const int64_t items = plan_items(p.groups, p.n_groups, p.L.Hq, STATS);
     if (items == 0) return SPAVA_OK;
     if (items >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
-    SPAVA_TRY(set_smem(attn_kernel<D, STATS>, SM::kAlloc));
-    attn_kernel<D, STATS><<<static_cast<unsigned>(items), kAttnThreads, SM::kAlloc, st>>>(p);
+    if (STATS) {
+        using SM = StatsSmem<D>;
+        SPAVA_TRY(set_smem(stats_kernel<D>, SM::kAlloc));
+        stats_kernel<D><<<static_cast<unsigned>(items), kStatsThreads, SM::kAlloc, st>>>(p);
+    } else {
+        using SM = AttnSmem<D>;
+        SPAVA_TRY(set_smem(attn_kernel<D>, SM::kAlloc));
+        attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, SM::kAlloc, st>>>(p);
+    }
     return launched();
 }
 

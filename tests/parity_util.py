@@ -104,18 +104,22 @@ def unique_mask(w: Workload, idx_gpu: np.ndarray, idx_ref: np.ndarray, rows, hea
     return ~context[:, None] | (v[:, None] <= first_diff[g_of][None, :])
 
 
-def check_convex(O_gpu: np.ndarray, V: torch.Tensor, heads, G: int, what=""):
+def check_convex(O_gpu: np.ndarray, V: torch.Tensor, heads, G: int, mask: np.ndarray, what=""):
     """Outputs whose key set is one of several valid ones: each is a softmax
     average of value rows of its KV group, so every coordinate lies within that
-    group's value range (plus bf16 rounding).  ``O_gpu[n, len(heads), d]``."""
+    group's value range (plus bf16 rounding).  ``O_gpu[n, len(heads), d]``; the
+    entries where ``mask[n, len(heads)]`` is True are checked."""
     Vf = V.float()
     lo = Vf.amin(dim=0).cpu().numpy()        # [Hkv, d]
     hi = Vf.amax(dim=0).cpu().numpy()
     g_of = np.asarray(heads) // G
     slack = 2.0 ** -7 * np.maximum(np.abs(lo), np.abs(hi))
-    assert np.isfinite(O_gpu).all(), f"{what}: non-finite output"
-    assert (O_gpu >= (lo - slack)[g_of][None]).all(), f"{what}: below the value range"
-    assert (O_gpu <= (hi + slack)[g_of][None]).all(), f"{what}: above the value range"
+    lo_e = np.broadcast_to((lo - slack)[g_of][None], O_gpu.shape)[mask]
+    hi_e = np.broadcast_to((hi + slack)[g_of][None], O_gpu.shape)[mask]
+    got = O_gpu[mask]
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    assert (got >= lo_e).all(), f"{what}: below the value range"
+    assert (got <= hi_e).all(), f"{what}: above the value range"
 
 
 def check_outputs(O_gpu: np.ndarray, O_ref: np.ndarray, what=""):

@@ -69,7 +69,7 @@ def test_full_size_layer(name):
     uniq = unique_mask(w, idx_h, idx_ref, rows, heads)
     assert uniq.mean() > 0.5
     mx, mean = check_outputs(O_got[uniq], O_ref[uniq], name)
-    check_convex(O_got[~uniq], V, heads, G, name)
+    check_convex(O_got, V, heads, G, ~uniq, name)
     lse_got = to_np(lse[heads][:, torch.from_numpy(rows).cuda()]).T
     np.testing.assert_allclose(lse_got[uniq], lse_ref[uniq], atol=LSE_ABS, rtol=0)
     print(f"{name}: selections exact {n_exact}, in-band {n_band}; O max {mx:.2e} mean {mean:.2e};"

@@ -147,7 +147,7 @@ def test_prefill_end_to_end(name):
     assert uniq.mean() > 0.5
     O_np = to_np(O)
     check_outputs(O_np[uniq], O_ref[uniq], name)
-    check_convex(O_np[~uniq], V, heads, w.Hq // w.Hkv, name)
+    check_convex(O_np, V, heads, w.Hq // w.Hkv, ~uniq, name)
     np.testing.assert_allclose(to_np(lse).T[uniq], lse_ref[uniq], atol=LSE_ABS, rtol=0)
 
 

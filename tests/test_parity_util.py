@@ -26,9 +26,18 @@ def test_unique_mask_marks_later_chunks_of_that_group():
 
 
 def test_check_convex_bounds():
-    V = torch.tensor([[[0.0, -1.0]], [[2.0, 1.0]]])      # [N=2, Hkv=1, d=2]
-    check_convex(np.array([[[1.0, 0.0], [2.0, -1.0]]]), V, [0, 0], 2)
+    # two KV groups with different ranges; heads 0, 1 -> group 0, heads 2, 3 -> group 1
+    V = torch.tensor([[[0.0, -1.0], [10.0, 10.0]], [[2.0, 1.0], [12.0, 11.0]]])  # [N, Hkv, d]
+    O = np.array([[[1.0, 0.0], [2.0, -1.0], [11.0, 10.5], [12.0, 11.0]]])     # [1, 4 heads, d]
+    everything = np.ones((1, 4), dtype=bool)
+    check_convex(O, V, [0, 1, 2, 3], 2, everything)
+    bad = O.copy()
+    bad[0, 2, 0] = 2.5                    # inside group 0's range, below group 1's
     with pytest.raises(AssertionError):
-        check_convex(np.array([[[2.5, 0.0]]]), V, [0], 2)
+        check_convex(bad, V, [0, 1, 2, 3], 2, everything)
+    skip = everything.copy()
+    skip[0, 2] = False                    # entries outside the mask are not checked
+    check_convex(bad, V, [0, 1, 2, 3], 2, skip)
+    bad[0, 0, 1] = np.nan
     with pytest.raises(AssertionError):
-        check_convex(np.array([[[np.nan, 0.0]]]), V, [0], 2)
+        check_convex(bad, V, [0, 1, 2, 3], 2, skip)
