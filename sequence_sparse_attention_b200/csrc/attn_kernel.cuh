@@ -17,7 +17,7 @@
 //              conditional rescaling (the running max only moves when it grows
 //              by more than 2^8), P written back into TMEM as bf16.
 //   warp  8    TMA producer: Q_A, Q_B once, then K (one tile ahead) and V rings
-//   warp  9    MMA issuer, per key tile j:
+//   warp  9    MMA issuer (warps 10-11 only complete its warpgroup), per key tile j:
 //                PV_A(j)  S_A(j+1)  PV_B(j)  S_B(j+1)
 //              so S_X(j+1) enters the tensor pipe right behind PV_X(j) while the
 //              other tile's softmax is running.
@@ -73,10 +73,19 @@ struct AttnSmem {
 static_assert(AttnSmem<128>::kAlloc <= kMaxDynSmem, "attention smem over budget");
 static_assert(AttnSmem<64>::kAlloc <= kMaxDynSmem, "attention smem over budget");
 
+// Three warpgroups: softmax of tile A, softmax of tile B, and one holding the
+// TMA producer and the MMA issuer (its other two warps idle).  The third gives
+// registers to the first two: launched at kLaunchRegs per thread, it drops to
+// kRegsIo and the softmax warpgroups rise to kRegsSoftmax.
 constexpr int kSoftWarps = 8;  // 4 per query tile
-constexpr int kAttnThreads = (kSoftWarps + 2) * 32;
+constexpr int kAttnThreads = 3 * 128;
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
+constexpr int kLaunchRegs = 168;  // 65536 / 384, rounded down to the allocation unit of 8
+constexpr int kRegsIo = 80;
+constexpr int kRegsSoftmax = 208;
+static_assert(128 * kRegsIo + 256 * kRegsSoftmax <= kAttnThreads * kLaunchRegs,
+              "register split above the CTA's pool");
 constexpr int kColO = 256;  // O_A; O_B at kColO + 128
 
 // Work item = row tiles 2p and 2p+1 of a region.  Inside a group: KV head by KV
@@ -187,7 +196,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     const uint32_t tmem = *tmem_slot;
     const AbortState ab{abort_flag, P.status};
 
-    if (warp == kProducerWarp) {
+    if (warp >= kSoftWarps) {
+        reg_dealloc<kRegsIo>();
+        if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             mbar_expect_tx(q_full, hasB ? 2 * SM::kTile : SM::kTile);
@@ -327,7 +338,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
             mbar_wait_drain(mma_drain, 0);
         }
         __syncwarp();
+        }
     } else {
+        reg_alloc<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax
         const int x = warp >> 2, quarter = warp & 3;
         const int TX = x ? TB : TA;

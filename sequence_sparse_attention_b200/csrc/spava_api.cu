@@ -238,6 +238,11 @@ spava_status launch_attn(AttnParams &p, cudaStream_t st) {
         stats_kernel<D><<<static_cast<unsigned>(items), kStatsThreads, SM::kAlloc, st>>>(p);
     } else {
         using SM = AttnSmem<D>;
+        // The kernel's register split draws on the pool its launch allocates;
+        // refuse to launch a build whose per-thread count would leave it short.
+        cudaFuncAttributes fa;
+        SPAVA_CUDA(cudaFuncGetAttributes(&fa, attn_kernel<D>));
+        if (fa.numRegs < kLaunchRegs) return SPAVA_ERR_UNSUPPORTED;
         SPAVA_TRY(set_smem(attn_kernel<D>, SM::kAlloc));
         attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, SM::kAlloc, st>>>(p);
     }
