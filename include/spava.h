@@ -132,13 +132,23 @@ spava_status spava_prefill_attention(const spava_config *cfg, const void *q, con
 
 /* spava_prefill_attention from HOST buffers: copies q_host, k_host, v_host
  * into the caller's device buffers q, k, v, runs the layer, and copies o (and
- * lse if both lse and lse_host are non-NULL) back to o_host / lse_host, all
- * ordered on `stream`.  Host buffers should be page-locked for the copies to be
- * asynchronous; the call does not wait for them. */
+ * lse if both lse and lse_host are non-NULL) back to o_host / lse_host.
+ * Host buffers should be page-locked for the copies to be asynchronous; the
+ * call does not wait for them.
+ * copy_stream NULL (or equal to stream): everything is ordered on `stream`.
+ * Otherwise the copies run on copy_stream, overlapped with the kernels on
+ * `stream`: K, V and the query block's Q rows go up first (all that scoring
+ * needs), then V; the attention then runs in up to 8 groups of whole regions
+ * (the query block, then chunks and anchor in descending token order, costliest
+ * first), each starting once its Q rows have arrived, and each group's O (and
+ * lse) rows go down while later groups compute.  `stream` is made to wait for the last copy, so the call's work is
+ * complete when `stream` is.  The call creates and destroys its own CUDA events
+ * (no memory).  Neither stream may be capturing a graph. */
 spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q_host,
                                           const void *k_host, const void *v_host, void *o_host,
                                           float *lse_host, void *q, void *k, void *v, void *o,
-                                          float *lse, void *ws, size_t ws_bytes, void *stream);
+                                          float *lse, void *ws, size_t ws_bytes, void *stream,
+                                          void *copy_stream);
 
 /* Synchronises `stream`, reads the workspace status word (bit 0: a bounded wait
  * in a kernel gave up), writes it to *flags and clears it.  Returns

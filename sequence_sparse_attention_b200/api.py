@@ -173,11 +173,15 @@ class Spava:
                     _ptr(lse), _ptr(idx_out), _ptr(self.ws), self.ws.numel(), _stream(self.device))
         return o, lse, idx_out
 
-    def prefill_attention_host(self, q_host, k_host, v_host, o_host, lse_host, q, k, v, o, lse):
-        """Host (pinned) buffers in and out; device buffers are the caller's."""
+    def prefill_attention_host(self, q_host, k_host, v_host, o_host, lse_host, q, k, v, o, lse,
+                               copy_stream=None):
+        """Host (pinned) buffers in and out; device buffers are the caller's.
+        With a ``torch.cuda.Stream`` as ``copy_stream`` the copies overlap the
+        kernels (run on the current stream) group by group."""
+        cs = copy_stream.cuda_stream if copy_stream is not None else None
         native.call("spava_prefill_attention_host", self._args(), _ptr(q_host), _ptr(k_host),
                     _ptr(v_host), _ptr(o_host), _ptr(lse_host), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
-                    _ptr(lse), _ptr(self.ws), self.ws.numel(), _stream(self.device))
+                    _ptr(lse), _ptr(self.ws), self.ws.numel(), _stream(self.device), cs)
 
     def device_status(self) -> int:
         """Synchronises, returns and clears the kernels' status word (0 = clean)."""

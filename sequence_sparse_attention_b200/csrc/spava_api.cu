@@ -94,11 +94,25 @@ int item_tiles(const Layer &L, const Item &it) {
 // longest-processing-time-first schedule over the SMs.  Inside a group, items
 // run KV head by KV head, row tile descending, with the query heads of a KV
 // head adjacent (shared K/V tiles in L2; see decode_item).
-int plan_attention(const Layer &L, bool stats, Group *out) {
+// Rows of the region a group covers.
+void region_rows(const Layer &L, int kind, int sub, int &lo, int &hi) {
+    Item it{kind, sub, 0, 0};
+    int r0, re;
+    item_rows(L, it, r0, re);
+    lo = r0;
+    hi = kind == kCtx ? L.off[sub + 1] : kind == kAnchor ? L.a : L.N;
+}
+
+// Only regions lying inside rows [row_lo, row_hi) are planned (the whole layer
+// by default).
+int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int row_hi = INT32_MAX) {
     struct G { Group g; int cost; };
     std::vector<G> gs;
     auto push = [&](int kind, int sub, int n_rt) {
         if (n_rt <= 0) return;
+        int lo, hi;
+        region_rows(L, kind, sub, lo, hi);
+        if (lo < row_lo || hi > row_hi) return;
         Item it{kind, sub, n_rt - 1, 0};
         gs.push_back({Group{kind, sub, n_rt, 0}, item_tiles(L, it)});
     };
@@ -321,7 +335,8 @@ spava_status run_pack(const Layer &L, const void *k, const void *v, const int32_
 }
 
 spava_status run_attn(const Layer &L, const void *q, const void *k, const void *v, const void *pk,
-                      const void *pv, void *o, float *lse, char *ws, cudaStream_t st) {
+                      const void *pv, void *o, float *lse, char *ws, cudaStream_t st,
+                      int row_lo = 0, int row_hi = INT32_MAX) {
     const WsLayout w = ws_layout(L);
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
@@ -332,13 +347,14 @@ spava_status run_attn(const Layer &L, const void *q, const void *k, const void *
     // With no packed rows (a = 0, l = 0) no segment reads the packed maps.
     SPAVA_TRY(L.L > 0 ? map_packed(&p.tmPK, pk, L) : map_tokens(&p.tmPK, k, L, L.Hkv));
     SPAVA_TRY(L.L > 0 ? map_packed(&p.tmPV, pv, L) : map_tokens(&p.tmPV, v, L, L.Hkv));
-    p.n_groups = plan_attention(L, false, p.groups);
+    p.n_groups = plan_attention(L, false, p.groups, row_lo, row_hi);
     p.O = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     p.part_O = reinterpret_cast<float *>(ws + w.part_o);
     p.part_lse = reinterpret_cast<float *>(ws + w.part_lse);
     p.status = reinterpret_cast<int *>(ws + w.status);
     SPAVA_TRY(L.d == 128 ? launch_attn<128, false>(p, st) : launch_attn<64, false>(p, st));
+    if (L.N - L.q < row_lo || L.N > row_hi) return SPAVA_OK;  // query block not in this range
     const int64_t warps = static_cast<int64_t>(L.Hq) * L.q;
     const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
     auto O = static_cast<__nv_bfloat16 *>(o);
@@ -347,6 +363,56 @@ spava_status run_attn(const Layer &L, const void *q, const void *k, const void *
     else
         merge_kernel<64><<<blocks, 256, 0, st>>>(L, p.part_O, p.part_lse, O, lse);
     return launched();
+}
+
+// Scoring, selection and gather: everything of the layer before the attention.
+spava_status run_front(const Layer &L, const void *q, const void *k, const void *v,
+                       int32_t *idx_out, char *w, cudaStream_t st) {
+    const WsLayout lay = ws_layout(L);
+    float *scores = reinterpret_cast<float *>(w + lay.scores);
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + lay.idx);
+    if (L.n_chunks > 1 && L.l > 0) {
+        SPAVA_TRY(run_stats(L, q, k, w, st));
+        SPAVA_TRY(run_scores(L, q, k, scores, w, st));
+        SPAVA_TRY(run_topk(L, scores, idx, st));
+    }
+    return run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st);
+}
+
+// Row groups of the copy/compute pipeline of the host entry point, in the
+// order they run: the query block first (its Q rows go up with K, ahead of
+// everything else), then the chunks and the anchor in DESCENDING token order.
+// Later chunks attend more keys, so the first context groups bring the most
+// work per uploaded row and the copies run ahead of the kernels; the last
+// group, whose download no kernel hides, is the first region alone (the
+// cheapest).  The last chunk is alone too; the regions between are cut into
+// runs of about equal rows.  Group g covers rows [lo[g], hi[g]); returns the
+// count (at most kCopyGroups).
+constexpr int kCopyGroups = 8;
+int copy_groups(const Layer &L, int *lo, int *hi) {
+    std::vector<int> starts;  // starts of the anchor and chunk regions, in token order
+    if (L.a > 0) starts.push_back(0);
+    for (int v = 0; v < L.n_chunks; ++v) starts.push_back(L.off[v]);
+    const int ctx_end = L.N - L.q;
+    int n = 0;
+    lo[n] = ctx_end, hi[n++] = L.N;
+    const int m = static_cast<int>(starts.size());
+    lo[n] = starts[m - 1], hi[n++] = ctx_end;  // the last chunk
+    if (m == 1) return n;
+    // regions m-2 .. 1 (descending), then region 0 alone
+    const int mid_hi = starts[m - 1], mid_lo = starts[1];
+    const int mid_groups = kCopyGroups - 3;
+    int end = mid_hi;
+    for (int i = m - 2; i >= 1; --i) {
+        const int64_t k = n - 1;  // middle groups cut so far + 1
+        const int64_t target = mid_hi - static_cast<int64_t>(mid_hi - mid_lo) * k / mid_groups;
+        if (starts[i] <= target || i == 1) {
+            lo[n] = starts[i], hi[n++] = end;
+            end = starts[i];
+        }
+    }
+    lo[n] = 0, hi[n++] = starts[1];
+    return n;
 }
 
 }  // namespace
@@ -439,24 +505,16 @@ spava_status spava_prefill_attention(const spava_config *cfg, const void *q, con
     SPAVA_TRY(check_ws(L, ws, ws_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *w = static_cast<char *>(ws);
+    SPAVA_TRY(run_front(L, q, k, v, idx_out, w, st));
     const WsLayout lay = ws_layout(L);
-    float *scores = reinterpret_cast<float *>(w + lay.scores);
-    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + lay.idx);
-    void *pk = w + lay.pk;
-    void *pv = w + lay.pv;
-    if (L.n_chunks > 1 && L.l > 0) {
-        SPAVA_TRY(run_stats(L, q, k, w, st));
-        SPAVA_TRY(run_scores(L, q, k, scores, w, st));
-        SPAVA_TRY(run_topk(L, scores, idx, st));
-    }
-    SPAVA_TRY(run_pack(L, k, v, idx, pk, pv, st));
-    return run_attn(L, q, k, v, pk, pv, o, lse, w, st);
+    return run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st);
 }
 
 spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q_host,
                                           const void *k_host, const void *v_host, void *o_host,
                                           float *lse_host, void *q, void *k, void *v, void *o,
-                                          float *lse, void *ws, size_t ws_bytes, void *stream) {
+                                          float *lse, void *ws, size_t ws_bytes, void *stream,
+                                          void *copy_stream) {
     Layer L;
     SPAVA_TRY(make_layer(cfg, &L));
     if (!q_host || !k_host || !v_host || !o_host) return SPAVA_ERR_INVALID_ARG;
@@ -464,20 +522,89 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
     SPAVA_TRY(check_ptr(k));
     SPAVA_TRY(check_ptr(v));
     SPAVA_TRY(check_ptr(o));
+    SPAVA_TRY(check_ptr(lse, false));
     SPAVA_TRY(check_ws(L, ws, ws_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t qb = size_t(L.N) * L.Hq * L.d * 2, kb = size_t(L.N) * L.Hkv * L.d * 2;
-    SPAVA_CUDA(cudaMemcpyAsync(q, q_host, qb, cudaMemcpyHostToDevice, st));
-    SPAVA_CUDA(cudaMemcpyAsync(k, k_host, kb, cudaMemcpyHostToDevice, st));
-    SPAVA_CUDA(cudaMemcpyAsync(v, v_host, kb, cudaMemcpyHostToDevice, st));
+    const size_t row_q = size_t(L.Hq) * L.d * 2, row_k = size_t(L.Hkv) * L.d * 2;
     const bool want_lse = lse && lse_host;
-    SPAVA_TRY(spava_prefill_attention(cfg, q, k, v, o, want_lse ? lse : nullptr, nullptr, ws,
-                                      ws_bytes, stream));
-    SPAVA_CUDA(cudaMemcpyAsync(o_host, o, qb, cudaMemcpyDeviceToHost, st));
-    if (want_lse)
-        SPAVA_CUDA(cudaMemcpyAsync(lse_host, lse, sizeof(float) * size_t(L.Hq) * L.N,
-                                   cudaMemcpyDeviceToHost, st));
-    return SPAVA_OK;
+    auto cq = static_cast<const char *>(q_host);
+    auto oh = static_cast<char *>(o_host);
+    char *qd = static_cast<char *>(q), *od = static_cast<char *>(o);
+    auto d2h_rows = [&](int r0, int r1, cudaStream_t s) -> spava_status {
+        SPAVA_CUDA(cudaMemcpyAsync(oh + r0 * row_q, od + r0 * row_q, (r1 - r0) * row_q,
+                                   cudaMemcpyDeviceToHost, s));
+        if (want_lse)  // lse is [Hq, N]: the rows of every head, one strided copy
+            SPAVA_CUDA(cudaMemcpy2DAsync(lse_host + r0, sizeof(float) * L.N, lse + r0,
+                                         sizeof(float) * L.N, sizeof(float) * (r1 - r0), L.Hq,
+                                         cudaMemcpyDeviceToHost, s));
+        return SPAVA_OK;
+    };
+    if (!copy_stream || copy_stream == stream) {
+        SPAVA_CUDA(cudaMemcpyAsync(q, q_host, L.N * row_q, cudaMemcpyHostToDevice, st));
+        SPAVA_CUDA(cudaMemcpyAsync(k, k_host, L.N * row_k, cudaMemcpyHostToDevice, st));
+        SPAVA_CUDA(cudaMemcpyAsync(v, v_host, L.N * row_k, cudaMemcpyHostToDevice, st));
+        SPAVA_TRY(spava_prefill_attention(cfg, q, k, v, o, want_lse ? lse : nullptr, nullptr, ws,
+                                          ws_bytes, stream));
+        return d2h_rows(0, L.N, st);
+    }
+    // Pipelined: K and the query block's Q rows (all that scoring needs) go up
+    // first, then V (the gather needs it), then the Q rows of each context
+    // group; the attention runs group by group as its Q rows arrive, and each
+    // group's O goes down while later groups compute.
+    cudaStream_t cs = static_cast<cudaStream_t>(copy_stream);
+    int lo[kCopyGroups], hi[kCopyGroups];
+    const int ng = copy_groups(L, lo, hi);
+    std::vector<cudaEvent_t> ev(2 * ng + 3, nullptr);  // front, V, Q of each group, attention, done
+    spava_status rc = SPAVA_OK;
+    for (auto &e : ev)
+        if (rc == SPAVA_OK && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
+            rc = cuda_fail(cudaGetLastError());
+    auto body = [&]() -> spava_status {
+        cudaEvent_t e_front = ev[0], e_v = ev[1], *e_q = &ev[2], *e_a = &ev[2 + ng], e_done = ev[2 + 2 * ng];
+        SPAVA_CUDA(cudaMemcpyAsync(k, k_host, L.N * row_k, cudaMemcpyHostToDevice, cs));
+        SPAVA_CUDA(cudaMemcpyAsync(qd + lo[0] * row_q, cq + lo[0] * row_q, (hi[0] - lo[0]) * row_q,
+                                   cudaMemcpyHostToDevice, cs));
+        SPAVA_CUDA(cudaEventRecord(e_front, cs));
+        SPAVA_CUDA(cudaMemcpyAsync(v, v_host, L.N * row_k, cudaMemcpyHostToDevice, cs));
+        SPAVA_CUDA(cudaEventRecord(e_v, cs));
+        for (int g = 1; g < ng; ++g) {
+            SPAVA_CUDA(cudaMemcpyAsync(qd + lo[g] * row_q, cq + lo[g] * row_q, (hi[g] - lo[g]) * row_q,
+                                       cudaMemcpyHostToDevice, cs));
+            SPAVA_CUDA(cudaEventRecord(e_q[g], cs));
+        }
+        char *w = static_cast<char *>(ws);
+        const WsLayout lay = ws_layout(L);
+        const WsLayout &wl = lay;
+        float *scores = reinterpret_cast<float *>(w + wl.scores);
+        int32_t *idx = reinterpret_cast<int32_t *>(w + wl.idx);
+        SPAVA_CUDA(cudaStreamWaitEvent(st, e_front, 0));
+        if (L.n_chunks > 1 && L.l > 0) {
+            SPAVA_TRY(run_stats(L, q, k, w, st));
+            SPAVA_TRY(run_scores(L, q, k, scores, w, st));
+            SPAVA_TRY(run_topk(L, scores, idx, st));
+        }
+        SPAVA_CUDA(cudaStreamWaitEvent(st, e_v, 0));
+        SPAVA_TRY(run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st));
+        for (int g = 0; g < ng; ++g) {
+            if (g > 0) SPAVA_CUDA(cudaStreamWaitEvent(st, e_q[g], 0));
+            SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, want_lse ? lse : nullptr, w,
+                               st, lo[g], hi[g]));
+            SPAVA_CUDA(cudaEventRecord(e_a[g], st));
+        }
+        for (int g = 0; g < ng; ++g) {
+            SPAVA_CUDA(cudaStreamWaitEvent(cs, e_a[g], 0));
+            SPAVA_TRY(d2h_rows(lo[g], hi[g], cs));
+        }
+        // The call's work ends on `stream`, after the last copy.
+        SPAVA_CUDA(cudaEventRecord(e_done, cs));
+        SPAVA_CUDA(cudaStreamWaitEvent(st, e_done, 0));
+        return SPAVA_OK;
+    };
+    if (rc == SPAVA_OK) rc = body();
+    // Destroying a recorded event is safe: its resources go once it completes.
+    for (auto e : ev)
+        if (e) cudaEventDestroy(e);
+    return rc;
 }
 
 spava_status spava_device_status(void *ws, size_t ws_bytes, void *stream, int32_t *flags) {

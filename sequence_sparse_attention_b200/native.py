@@ -70,7 +70,7 @@ def load() -> ctypes.CDLL:
         "spava_pack_passing": [cfgp, vp, vp, vp, vp, vp, vp],
         "spava_attn": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "spava_prefill_attention": [cfgp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
-        "spava_prefill_attention_host": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "spava_prefill_attention_host": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp],
         "spava_device_status": [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)],
         "spava_attended_pairs": [cfgp, i64p, i64p],
         "spava_score_noalloc": [cfgp, vp, vp, vp, vp],

@@ -177,19 +177,27 @@ def test_repeat_calls_bit_identical():
     assert torch.equal(l1, l2)
 
 
-def test_host_buffers_entry_point():
-    w = CASES["tiny"]
+@pytest.mark.parametrize("name", ["tiny", "g7", "no_anchor", "long_anchor", "short_chunks"])
+@pytest.mark.parametrize("pipelined", [False, True])
+def test_host_buffers_entry_point(name, pipelined):
+    """Host buffers in and out, on one stream or with the copies on a second
+    stream overlapping the kernels group by group: bit-identical to the
+    device-buffer entry point."""
+    w = CASES[name]
     Q, K, V, _ = make_inputs(w)
     sp = Spava(Layout.from_workload(w))
     qh, kh, vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
-    oh = torch.empty_like(Q).pin_memory()
-    lh = torch.empty((w.Hq, w.N), dtype=torch.float32).pin_memory()
+    oh = torch.full_like(Q, 7.0).pin_memory()
+    lh = torch.full((w.Hq, w.N), 7.0, dtype=torch.float32).pin_memory()
     qd, kd, vd = torch.empty_like(Q, device="cuda"), torch.empty_like(K, device="cuda"), torch.empty_like(V, device="cuda")
     od = torch.empty_like(qd)
     ld = torch.empty((w.Hq, w.N), dtype=torch.float32, device="cuda")
-    sp.prefill_attention_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld)
+    cs = torch.cuda.Stream() if pipelined else None
+    sp.prefill_attention_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, copy_stream=cs)
+    torch.cuda.current_stream().synchronize()   # the call's work ends on this stream
+    oh_c, lh_c = oh.clone(), lh.clone()
     torch.cuda.synchronize()
     device_clean(sp)
     O_dev, lse_dev, _ = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda())
-    assert torch.equal(oh.view(torch.int16), O_dev.cpu().view(torch.int16))
-    assert torch.equal(lh, lse_dev.cpu())
+    assert torch.equal(oh_c.view(torch.int16), O_dev.cpu().view(torch.int16))
+    assert torch.equal(lh_c, lse_dev.cpu())
