@@ -6,7 +6,7 @@
 //     S[g, j] = sum_{h in g} sum_{i in query block} exp2(x_{h,i,j} - lse2_{u,h,i}),
 //     x = scale*log2(e) * q_{h,i} . k_{g,j},
 // where lse2_{u,h,i} is the base-2 log-sum-exp of row (h, i) over chunk u (the
-// statistics pass, attn_kernel in STATS mode).  Equivalently: softmax over the
+// statistics pass, stats_kernel.cuh).  Equivalently: softmax over the
 // chunk, summed over query rows and group heads.
 //
 // One CTA = 128 keys of one chunk and one KV head.  The product is formed
