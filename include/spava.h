@@ -137,13 +137,17 @@ spava_status spava_prefill_attention(const spava_config *cfg, const void *q, con
  * call does not wait for them.
  * copy_stream NULL (or equal to stream): everything is ordered on `stream`.
  * Otherwise the copies run on copy_stream, overlapped with the kernels on
- * `stream`: K, V and the query block's Q rows go up first (all that scoring
+ * `stream`: K and the query block's Q rows go up first (all that scoring
  * needs), then V; the attention then runs in up to 8 groups of whole regions
  * (the query block, then chunks and anchor in descending token order, costliest
  * first), each starting once its Q rows have arrived, and each group's O (and
- * lse) rows go down while later groups compute.  `stream` is made to wait for the last copy, so the call's work is
- * complete when `stream` is.  The call creates and destroys its own CUDA events
- * (no memory).  Neither stream may be capturing a graph. */
+ * lse) rows go down while later groups compute.  The copies begin only after
+ * all work already enqueued on `stream` (an earlier call may still be reading
+ * the device buffers), and `stream` is made to wait for the last copy, so the
+ * call's work is complete when `stream` is and back-to-back calls on the same
+ * buffers stay ordered.  The call creates and destroys its own CUDA events (no
+ * memory).  Neither stream may be capturing a graph.  On an error return, work
+ * already enqueued may still run. */
 spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q_host,
                                           const void *k_host, const void *v_host, void *o_host,
                                           float *lse_host, void *q, void *k, void *v, void *o,

@@ -366,8 +366,10 @@ spava_status run_attn(const Layer &L, const void *q, const void *k, const void *
 }
 
 // Scoring, selection and gather: everything of the layer before the attention.
+// Scoring reads only K and the query block's Q rows; if `v_ready` is given, the
+// gather (the first step that reads V) waits for it.
 spava_status run_front(const Layer &L, const void *q, const void *k, const void *v,
-                       int32_t *idx_out, char *w, cudaStream_t st) {
+                       int32_t *idx_out, char *w, cudaStream_t st, cudaEvent_t v_ready = nullptr) {
     const WsLayout lay = ws_layout(L);
     float *scores = reinterpret_cast<float *>(w + lay.scores);
     int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + lay.idx);
@@ -376,6 +378,7 @@ spava_status run_front(const Layer &L, const void *q, const void *k, const void 
         SPAVA_TRY(run_scores(L, q, k, scores, w, st));
         SPAVA_TRY(run_topk(L, scores, idx, st));
     }
+    if (v_ready) SPAVA_CUDA(cudaStreamWaitEvent(st, v_ready, 0));
     return run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st);
 }
 
@@ -550,17 +553,23 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
     // Pipelined: K and the query block's Q rows (all that scoring needs) go up
     // first, then V (the gather needs it), then the Q rows of each context
     // group; the attention runs group by group as its Q rows arrive, and each
-    // group's O goes down while later groups compute.
+    // group's O goes down while later groups compute.  The copies start only
+    // once everything already on `stream` is done (an earlier call's kernels may
+    // still be reading the device buffers they overwrite).
     cudaStream_t cs = static_cast<cudaStream_t>(copy_stream);
     int lo[kCopyGroups], hi[kCopyGroups];
     const int ng = copy_groups(L, lo, hi);
-    std::vector<cudaEvent_t> ev(2 * ng + 3, nullptr);  // front, V, Q of each group, attention, done
+    // start, front, V, Q of groups 1.., attention of each group, done
+    std::vector<cudaEvent_t> ev(2 * ng + 4, nullptr);
     spava_status rc = SPAVA_OK;
     for (auto &e : ev)
         if (rc == SPAVA_OK && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
             rc = cuda_fail(cudaGetLastError());
     auto body = [&]() -> spava_status {
-        cudaEvent_t e_front = ev[0], e_v = ev[1], *e_q = &ev[2], *e_a = &ev[2 + ng], e_done = ev[2 + 2 * ng];
+        cudaEvent_t e_start = ev[0], e_front = ev[1], e_v = ev[2], *e_q = &ev[3], *e_a = &ev[3 + ng],
+                    e_done = ev[3 + 2 * ng];
+        SPAVA_CUDA(cudaEventRecord(e_start, st));
+        SPAVA_CUDA(cudaStreamWaitEvent(cs, e_start, 0));
         SPAVA_CUDA(cudaMemcpyAsync(k, k_host, L.N * row_k, cudaMemcpyHostToDevice, cs));
         SPAVA_CUDA(cudaMemcpyAsync(qd + lo[0] * row_q, cq + lo[0] * row_q, (hi[0] - lo[0]) * row_q,
                                    cudaMemcpyHostToDevice, cs));
@@ -574,17 +583,8 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
         }
         char *w = static_cast<char *>(ws);
         const WsLayout lay = ws_layout(L);
-        const WsLayout &wl = lay;
-        float *scores = reinterpret_cast<float *>(w + wl.scores);
-        int32_t *idx = reinterpret_cast<int32_t *>(w + wl.idx);
         SPAVA_CUDA(cudaStreamWaitEvent(st, e_front, 0));
-        if (L.n_chunks > 1 && L.l > 0) {
-            SPAVA_TRY(run_stats(L, q, k, w, st));
-            SPAVA_TRY(run_scores(L, q, k, scores, w, st));
-            SPAVA_TRY(run_topk(L, scores, idx, st));
-        }
-        SPAVA_CUDA(cudaStreamWaitEvent(st, e_v, 0));
-        SPAVA_TRY(run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st));
+        SPAVA_TRY(run_front(L, q, k, v, nullptr, w, st, e_v));
         for (int g = 0; g < ng; ++g) {
             if (g > 0) SPAVA_CUDA(cudaStreamWaitEvent(st, e_q[g], 0));
             SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, want_lse ? lse : nullptr, w,

@@ -3,6 +3,8 @@ element, on sizes the oracle finishes in seconds that still span several 128
 tiles and ragged tails (chunk, anchor and query lengths not multiples of 128,
 GQA groups of 2 and 7, d = 64 and 128, uneven chunks, a = 0, one host, full
 passing blocks, local_pair_full = 0)."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -201,3 +203,28 @@ def test_host_buffers_entry_point(name, pipelined):
     O_dev, lse_dev, _ = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda())
     assert torch.equal(oh_c.view(torch.int16), O_dev.cpu().view(torch.int16))
     assert torch.equal(lh_c, lse_dev.cpu())
+
+
+def test_host_buffers_back_to_back():
+    """Two pipelined host calls in a row on the same device buffers with
+    different inputs: the second call's uploads must wait for the first call's
+    kernels, so each host output matches the device path for its own inputs."""
+    w = WORKLOADS["16k"]
+    ins = [make_inputs(w), make_inputs(dataclasses.replace(w, seed=w.seed + 100))]
+    sp = Spava(Layout.from_workload(w))
+    qd = torch.empty(ins[0][0].shape, dtype=torch.bfloat16, device="cuda")
+    kd = torch.empty(ins[0][1].shape, dtype=torch.bfloat16, device="cuda")
+    vd = torch.empty_like(kd)
+    od = torch.empty_like(qd)
+    cs = torch.cuda.Stream()
+    outs = []
+    hosts = []
+    for Q, K, V, _ in ins:
+        hosts.append((Q.pin_memory(), K.pin_memory(), V.pin_memory(), torch.empty_like(Q).pin_memory()))
+    for qh, kh, vh, oh in hosts:
+        sp.prefill_attention_host(qh, kh, vh, oh, None, qd, kd, vd, od, None, copy_stream=cs)
+    torch.cuda.synchronize()
+    device_clean(sp)
+    for (Q, K, V, _), (_, _, _, oh) in zip(ins, hosts):
+        O_dev, _, _ = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda())
+        assert torch.equal(oh.view(torch.int16), O_dev.cpu().view(torch.int16))
