@@ -47,6 +47,8 @@ struct AttnParams {
     float *part_lse;    // [2H+2, Hq, q] log2 domain
     float *stats;       // [2H-1, Hq, q] log2-domain lse of the query rows per chunk
     int *status;        // workspace status word
+    int *queue;         // work-item counter of the persistent attention grid (zeroed per launch)
+    int32_t n_items;    // work items of the attention launch
 };
 
 // sm_100 allows at most 227 KiB of dynamic shared memory per CTA.
@@ -87,6 +89,7 @@ constexpr int kRegsSoftmax = 208;
 static_assert(128 * kRegsIo + 256 * kRegsSoftmax <= kAttnThreads * kLaunchRegs,
               "register split above the CTA's pool");
 constexpr int kColO = 256;  // O_A; O_B at kColO + 128
+constexpr int kItemBar = 1;  // named barrier of all threads between work items
 
 // Work item = row tiles 2p and 2p+1 of a region.  Inside a group: KV head by KV
 // head, pairs in descending cost, the query heads of a KV head adjacent.
@@ -122,6 +125,33 @@ __device__ __forceinline__ float max128(const float (&x)[128]) {
     return fmaxf(fmax3(m[0], m[1], m[2]), m[3]);
 }
 
+// Everything about work item b that the roles need: rows of tiles A and B, the
+// key segments and tile counts.
+struct ItemPlan {
+    Item it;
+    int r0A, eA, r0B, eB;
+    bool hasB;
+    Seg segs[kMaxSegs];
+    int ns, T, TA, TB, g;
+};
+
+__device__ __forceinline__ void plan_item(const Layer &L, const Group *groups, int n_groups, int b,
+                                          ItemPlan &ip) {
+    ip.it = decode_pair_item(groups, n_groups, b, L.G);
+    Item it_b = ip.it;
+    it_b.rt = ip.it.rt + 1;
+    item_rows(L, ip.it, ip.r0A, ip.eA);
+    item_rows(L, it_b, ip.r0B, ip.eB);
+    ip.hasB = ip.eB > ip.r0B;
+    ip.ns = build_segments(L, ip.hasB ? it_b : ip.it, ip.segs);
+    ip.T = count_tiles(ip.segs, ip.ns);
+    // A causal last segment starts on a tile boundary of the region, so its last
+    // tile for B is B's diagonal, which lies beyond every row of A.
+    ip.TA = (ip.hasB && ip.ns > 0 && ip.segs[ip.ns - 1].causal) ? ip.T - 1 : ip.T;
+    ip.TB = ip.hasB ? ip.T : 0;
+    ip.g = ip.it.h / L.G;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
     using SM = AttnSmem<D>;
@@ -147,40 +177,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Layer &L = P.L;
-    const Item it = decode_pair_item(P.groups, P.n_groups, blockIdx.x, L.G);
-    Item it_b = it;
-    it_b.rt = it.rt + 1;
-    int r0A, eA, r0B, eB;
-    item_rows(L, it, r0A, eA);
-    item_rows(L, it_b, r0B, eB);
-    const bool hasB = eB > r0B;
-    Seg segs[kMaxSegs];
-    const int ns = build_segments(L, hasB ? it_b : it, segs);
-    const int T = count_tiles(segs, ns);
-    // A causal last segment starts on a tile boundary of the region, so its last
-    // tile for B is B's diagonal, which lies beyond every row of A.
-    const int TA = (hasB && ns > 0 && segs[ns - 1].causal) ? T - 1 : T;
-    const int TB = hasB ? T : 0;
-    const int g = it.h / L.G;
+    int *claim = reinterpret_cast<int *>(smem + SM::kOffMisc + 8);
 
-    if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
+    // Barriers start every item fresh: between items (nothing in flight any
+    // more) they are invalidated and initialised again.
+    auto init_bars = [&](bool again) {
+        auto init = [&](uint64_t *bar, uint32_t count) {
+            if (again) mbar_inval(bar);
+            mbar_init(bar, count);
+        };
+        init(q_full, 1);
         for (int i = 0; i < KS; ++i) {
-            mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 1);
+            init(&k_full[i], 1);
+            init(&k_empty[i], 1);
         }
         for (int i = 0; i < VS; ++i) {
-            mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 1);
+            init(&v_full[i], 1);
+            init(&v_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 128);
-            mbar_init(&o_done[i], 1);
+            init(&s_full[i], 1);
+            init(&p_full[i], 128);
+            init(&o_done[i], 1);
         }
-        mbar_init(mma_drain, 1);
-        *abort_flag = 0;
+        init(mma_drain, 1);
         fence_mbar_init();
+    };
+    if (threadIdx.x == 0) {
+        init_bars(false);
+        *abort_flag = 0;
     }
     if (warp == kProducerWarp && lane == 0) {
         tma_prefetch(&P.tmQ);
@@ -196,8 +221,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     const uint32_t tmem = *tmem_slot;
     const AbortState ab{abort_flag, P.status};
 
+    // Persistent grid: each CTA claims work items one at a time from a queue in
+    // the workspace, in the planner's order (costliest first), i.e. greedy
+    // longest-processing-time-first over the SMs.  The claim happens between two
+    // CTA-wide barriers, after every role is done with the previous item; a CTA
+    // whose waits gave up claims nothing more.
+    auto next_item = [&](int round) -> int {
+        if (threadIdx.x == kProducerWarp * 32) {
+            if (round > 0) init_bars(true);
+            *claim = *abort_flag ? INT32_MAX : atomicAdd(P.queue, 1);
+        }
+        tc_fence_before();
+        bar_sync(kItemBar, kAttnThreads);
+        tc_fence_after();
+        return *claim;
+    };
+    auto end_item = [&]() {
+        tc_fence_before();
+        bar_sync(kItemBar, kAttnThreads);
+        tc_fence_after();
+    };
+
     if (warp >= kSoftWarps) {
         reg_dealloc<kRegsIo>();
+        for (int round = 0;; ++round) {
+        const int b = next_item(round);
+        if (b >= P.n_items) break;
+        ItemPlan ip;
+        plan_item(L, P.groups, P.n_groups, b, ip);
+        const Item &it = ip.it;
+        const int r0A = ip.r0A, r0B = ip.r0B, T = ip.T, TA = ip.TA, TB = ip.TB, g = ip.g;
+        const bool hasB = ip.hasB;
+        const Seg *segs = ip.segs;
         if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -339,8 +394,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         }
         __syncwarp();
         }
+        end_item();
+        }
     } else {
         reg_alloc<kRegsSoftmax>();
+        for (int round = 0;; ++round) {
+        const int b = next_item(round);
+        if (b >= P.n_items) break;
+        ItemPlan ip;
+        plan_item(L, P.groups, P.n_groups, b, ip);
+        const Item &it = ip.it;
+        const int r0A = ip.r0A, r0B = ip.r0B, eA = ip.eA, eB = ip.eB, TA = ip.TA, TB = ip.TB;
+        const Seg *segs = ip.segs;
         // ------------------------------------------------------------ softmax
         const int x = warp >> 2, quarter = warp & 3;
         const int TX = x ? TB : TA;
@@ -481,6 +546,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                     if (valid && P.lse) P.lse[static_cast<size_t>(it.h) * L.N + t] = lse2 * 0.69314718055994531f;
                 }
             }
+        }
+        end_item();
         }
     }
 

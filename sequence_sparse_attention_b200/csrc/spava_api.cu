@@ -89,11 +89,6 @@ int item_tiles(const Layer &L, const Item &it) {
     return count_tiles(s, n);
 }
 
-// Groups of the attention launch, most expensive first: the hardware block
-// scheduler hands out CTAs in index order, so a cost-descending order is a
-// longest-processing-time-first schedule over the SMs.  Inside a group, items
-// run KV head by KV head, row tile descending, with the query heads of a KV
-// head adjacent (shared K/V tiles in L2; see decode_item).
 // Rows of the region a group covers.
 void region_rows(const Layer &L, int kind, int sub, int &lo, int &hi) {
     Item it{kind, sub, 0, 0};
@@ -103,8 +98,14 @@ void region_rows(const Layer &L, int kind, int sub, int &lo, int &hi) {
     hi = kind == kCtx ? L.off[sub + 1] : kind == kAnchor ? L.a : L.N;
 }
 
-// Only regions lying inside rows [row_lo, row_hi) are planned (the whole layer
-// by default).
+// Groups of the attention launch, most expensive first: the persistent
+// attention grid claims work items from a queue in index order (and the
+// hardware block scheduler hands out the statistics pass's CTAs in index
+// order), so a cost-descending order is a longest-processing-time-first
+// schedule over the SMs.  Inside a group, items run KV head by KV head, row
+// tile descending, with the query heads of a KV head adjacent (shared K/V tiles
+// in L2; see decode_pair_item and decode_item).  Only regions lying inside
+// rows [row_lo, row_hi) are planned (the whole layer by default).
 int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int row_hi = INT32_MAX) {
     struct G { Group g; int cost; };
     std::vector<G> gs;
@@ -252,13 +253,21 @@ spava_status launch_attn(AttnParams &p, cudaStream_t st) {
         stats_kernel<D><<<static_cast<unsigned>(items), kStatsThreads, SM::kAlloc, st>>>(p);
     } else {
         using SM = AttnSmem<D>;
+        // Persistent grid: one CTA per SM (the shared memory allows no more),
+        // each claiming items from the queue in the workspace.
+        int dev = 0, n_sm = 148;
+        SPAVA_CUDA(cudaGetDevice(&dev));
+        SPAVA_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+        p.n_items = static_cast<int32_t>(items);
+        SPAVA_CUDA(cudaMemsetAsync(p.queue, 0, sizeof(int), st));
         // The kernel's register split draws on the pool its launch allocates;
         // refuse to launch a build whose per-thread count would leave it short.
         cudaFuncAttributes fa;
         SPAVA_CUDA(cudaFuncGetAttributes(&fa, attn_kernel<D>));
         if (fa.numRegs < kLaunchRegs) return SPAVA_ERR_UNSUPPORTED;
         SPAVA_TRY(set_smem(attn_kernel<D>, SM::kAlloc));
-        attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, SM::kAlloc, st>>>(p);
+        const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, n_sm));
+        attn_kernel<D><<<grid, kAttnThreads, SM::kAlloc, st>>>(p);
     }
     return launched();
 }
@@ -353,6 +362,7 @@ spava_status run_attn(const Layer &L, const void *q, const void *k, const void *
     p.part_O = reinterpret_cast<float *>(ws + w.part_o);
     p.part_lse = reinterpret_cast<float *>(ws + w.part_lse);
     p.status = reinterpret_cast<int *>(ws + w.status);
+    p.queue = reinterpret_cast<int *>(ws + w.status + 128);  // inside the 256-byte status block
     SPAVA_TRY(L.d == 128 ? launch_attn<128, false>(p, st) : launch_attn<64, false>(p, st));
     if (L.N - L.q < row_lo || L.N > row_hi) return SPAVA_OK;  // query block not in this range
     const int64_t warps = static_cast<int64_t>(L.Hq) * L.q;
