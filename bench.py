@@ -42,8 +42,8 @@ KERNELS_PER_STEP = 6   # stats, scores, top-l, pack, attention, query merge
 # DRAM traffic of one attention launch on the 128K layer, from the single-pass
 # ncu capture summarised in profiles/ (dram__bytes_read.sum + dram__bytes_write.sum);
 # valid only while the sources that decide it are unchanged (KERNEL_FILES).
-PROFILED_TRAFFIC = {"kernel_sha256": "e891bfd8a1b9f6dffc6e9d03da8c167fe59a582ff46aece1f181f209a6b4b35e",
-                    "bytes_per_launch": 3035620608 + 1099370240, "workload": "128k",
+PROFILED_TRAFFIC = {"kernel_sha256": "455cfe8879c44f4c32fb09f8f2ee40d04b83e959342ba5ef4a3536baa0d34e3d",
+                    "bytes_per_launch": 3092664320 + 1211644672, "workload": "128k",
                     "source": "profiles/attn_kernel_128k_dram.md"}
 KERNEL_FILES = ("attn_kernel.cuh", "plan.cuh", "sm100.cuh")  # what decides the attention launch
 
