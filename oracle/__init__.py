@@ -48,7 +48,8 @@ class _Cfg(ctypes.Structure):
         ("d", ctypes.c_int32), ("N", ctypes.c_int64), ("a", ctypes.c_int64),
         ("q", ctypes.c_int64), ("off", ctypes.POINTER(ctypes.c_int64)),
         ("l", ctypes.c_int32), ("scale", ctypes.c_double),
-        ("local_pair_full", ctypes.c_int32),
+        ("local_pair_full", ctypes.c_int32), ("score_norm", ctypes.c_int32),
+        ("score_pool", ctypes.c_int32),
     ]
 
 
@@ -70,6 +71,9 @@ def _load():
         lib.oracle_prefill_rows.argtypes = [P(_Cfg), c_u16p, c_u16p, c_u16p, c_i32p, c_i64p,
                                             ctypes.c_int64, c_i32p, ctypes.c_int32, c_dp, c_dp]
         lib.oracle_pair.argtypes = [ctypes.c_int, ctypes.c_int]
+        lib.oracle_pool_sums.argtypes = [c_dp, ctypes.c_int64, ctypes.c_int32, c_dp]
+        lib.oracle_pool_sums_f32.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_int64,
+                                             ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -89,6 +93,8 @@ class Problem:
     l: int
     scale: float = 0.0
     local_pair_full: int = 1
+    score_norm: int = 0     # 0: softmax over the chunk; 1: over the row's whole key set
+    score_pool: int = 0     # 0/1: none; odd w >= 3: select on w-key window sums
     _keep: list = field(default_factory=list, repr=False)
 
     def c(self) -> _Cfg:
@@ -96,7 +102,8 @@ class Problem:
         self._keep = [off]
         return _Cfg(self.H, self.Hq, self.Hkv, self.d, self.N, self.a, self.q,
                     off.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), self.l,
-                    float(self.scale), int(self.local_pair_full))
+                    float(self.scale), int(self.local_pair_full), int(self.score_norm),
+                    int(self.score_pool))
 
     @property
     def n_chunks(self) -> int:
@@ -145,11 +152,44 @@ def select_top_l(S: np.ndarray, base: int, l: int) -> np.ndarray:
     return out
 
 
+def pool_sums(S: np.ndarray, w: int) -> np.ndarray:
+    """Window sums of the pooled-score variant, in the dtype of ``S`` (float64
+    or float32, the latter in the GPU's order and precision)."""
+    if S.dtype == np.float32:
+        S = np.ascontiguousarray(S)
+        out = np.empty_like(S)
+        fp = ctypes.POINTER(ctypes.c_float)
+        rc = _load().oracle_pool_sums_f32(S.ctypes.data_as(fp), len(S), int(w), out.ctypes.data_as(fp))
+    else:
+        S = np.ascontiguousarray(S, dtype=np.float64)
+        out = np.empty_like(S)
+        dp = ctypes.POINTER(ctypes.c_double)
+        rc = _load().oracle_pool_sums(S.ctypes.data_as(dp), len(S), int(w), out.ctypes.data_as(dp))
+    if rc != 0:
+        raise ValueError(f"oracle_pool_sums failed ({rc})")
+    return out
+
+
+def selection_scores(p: Problem, scores: np.ndarray) -> np.ndarray:
+    """The values the selection ranks: the scores, or with ``score_pool`` > 1
+    their window sums taken chunk by chunk."""
+    if p.score_pool <= 1:
+        return scores
+    out = np.array(scores, copy=True)
+    for u in range(p.n_chunks - 1):
+        s0, s1 = int(p.offsets[u] - p.a), int(p.offsets[u + 1] - p.a)
+        for g in range(out.shape[0]):
+            if not np.isnan(out[g, s0]):
+                out[g, s0:s1] = pool_sums(scores[g, s0:s1], p.score_pool)
+    return out
+
+
 def scores_and_select(p: Problem, Q: np.ndarray, K: np.ndarray, groups=None):
     """Scores and passing blocks of every producing chunk u < 2H-1.
 
     Returns ``(scores, idx)``: ``scores[g]`` is the float64 vector over the
-    context tokens (chunk u at ``offsets[u]-a``), ``idx`` is int32
+    context tokens (chunk u at ``offsets[u]-a``; raw scores, before any
+    pooling the selection applies), ``idx`` is int32
     ``[2H-1, Hkv, l]``.  KV heads not in ``groups`` are left as NaN / -2
     (not computed) so that a caller cannot use them by accident.
     """
@@ -162,7 +202,8 @@ def scores_and_select(p: Problem, Q: np.ndarray, K: np.ndarray, groups=None):
             S = chunk_scores(p, Q, K, u, g)
             s0 = int(p.offsets[u] - p.a)
             scores[g, s0:s0 + len(S)] = S
-            idx[u, g] = select_top_l(S, int(p.offsets[u]), p.l)
+            ranked = pool_sums(S, p.score_pool) if p.score_pool > 1 else S
+            idx[u, g] = select_top_l(ranked, int(p.offsets[u]), p.l)
     return scores, idx
 
 

@@ -50,6 +50,9 @@
  *   R10 inputs are post-rotary; kept keys keep their position.
  *   R11 scale = 1/sqrt(d) unless given; lse in natural log.
  *   R14 the last chunk produces no passing block (no successor).
+ *   Selection variants (ablations of R4, off by default): score_norm 1 takes
+ *   each query row's weights against its whole key set [0, t] instead of the
+ *   chunk alone; score_pool w ranks keys by w-key window sums of the scores.
  */
 #include <math.h>
 #include <stdint.h>
@@ -67,6 +70,8 @@ typedef struct {
     int32_t l;          /* passing-block size per KV head per chunk */
     double scale;       /* <= 0 means 1/sqrt(d) */
     int32_t local_pair_full;
+    int32_t score_norm; /* 0: softmax over the chunk (R4); 1: over the row's whole key set [0, t] */
+    int32_t score_pool; /* 0 or 1: none; odd w >= 3: rank by sums over w-key windows */
 } oracle_cfg;
 
 enum { ORACLE_OK = 0, ORACLE_EINVAL = -1, ORACLE_ENOMEM = -2 };
@@ -97,6 +102,8 @@ int oracle_validate(const oracle_cfg *c) {
     if (c->H < 1 || c->Hq < 1 || c->Hkv < 1 || c->d < 1) return ORACLE_EINVAL;
     if (c->Hq % c->Hkv) return ORACLE_EINVAL;
     if (c->a < 0 || c->q < 1 || c->l < 0) return ORACLE_EINVAL;
+    if (c->score_norm < 0 || c->score_norm > 1) return ORACLE_EINVAL;
+    if (c->score_pool < 0 || (c->score_pool > 1 && c->score_pool % 2 == 0)) return ORACLE_EINVAL;
     int nc = 2 * c->H;
     if (c->off[0] != c->a || c->off[nc] != c->N - c->q) return ORACLE_EINVAL;
     for (int v = 0; v < nc; ++v)
@@ -118,7 +125,9 @@ static double dot_bf16(const uint16_t *x, const uint16_t *y, int d) {
  * Passaggio"; reading R4):
  *   S[j] = sum_{h in g} sum_{i in query block} exp(x_{h,i,j} - m_{h,i}) / l_{h,i},
  *   x_{h,i,j} = scale * q_{h,i} . k_{g,j},  m, l the max and the sum of exp
- *   over j in chunk u only.
+ *   over j in chunk u only (score_norm 0), or over every key the row attends,
+ *   [0, t] with t = N - q + i (score_norm 1: the row's own attention weights,
+ *   the variant normalised by the query pass's log-sum-exp).
  * S has n_u = off[u+1]-off[u] entries, S[j - off[u]].
  * Step 1 computes (m, l) per query row; step 2 sums the probabilities per key
  * in a fixed (h, i) order, so the result does not depend on the thread count. */
@@ -139,14 +148,16 @@ int oracle_chunk_scores(const oracle_cfg *c, const uint16_t *Q, const uint16_t *
         const int h = g * G + (int)(r / c->q);
         const int64_t t = c->N - c->q + r % c->q;
         const uint16_t *qv = Q + ((size_t)t * c->Hq + h) * d;
+        /* normaliser's key range: the chunk, or everything the row attends */
+        const int64_t k0 = c->score_norm ? 0 : j0, k1 = c->score_norm ? t + 1 : j0 + n;
         double mx = -INFINITY;
-        for (int64_t j = 0; j < n; ++j) {
-            double x = sc * dot_bf16(qv, K + ((size_t)(j0 + j) * c->Hkv + g) * d, d);
+        for (int64_t j = k0; j < k1; ++j) {
+            double x = sc * dot_bf16(qv, K + ((size_t)j * c->Hkv + g) * d, d);
             if (x > mx) mx = x;
         }
         double sum = 0.0;
-        for (int64_t j = 0; j < n; ++j) {
-            double x = sc * dot_bf16(qv, K + ((size_t)(j0 + j) * c->Hkv + g) * d, d);
+        for (int64_t j = k0; j < k1; ++j) {
+            double x = sc * dot_bf16(qv, K + ((size_t)j * c->Hkv + g) * d, d);
             sum += exp(x - mx);
         }
         m[r] = mx;
@@ -167,6 +178,36 @@ int oracle_chunk_scores(const oracle_cfg *c, const uint16_t *Q, const uint16_t *
     }
     free(m);
     free(ls);
+    return ORACLE_OK;
+}
+
+/* Pooled-score variant of the selection (the pages name SnapKV's scoring only
+ * by title; the reading here: a window mean of w keys centred on each key,
+ * zero outside the chunk).  The mean divides every window by the same w, so
+ * ranking by it is ranking by the window SUM, which is what these return:
+ * out[j] = sum of S[j'] for j' in [j - w/2, j + w/2] clipped to [0, n), added
+ * in ascending j'.  w <= 1 copies S. */
+int oracle_pool_sums(const double *S, int64_t n, int32_t w, double *out) {
+    if (n < 0 || w < 0) return ORACLE_EINVAL;
+    const int64_t h = w > 1 ? w / 2 : 0;
+    for (int64_t j = 0; j < n; ++j) {
+        double s = 0.0;
+        for (int64_t k = (j - h < 0 ? 0 : j - h); k <= j + h && k < n; ++k) s += S[k];
+        out[j] = s;
+    }
+    return ORACLE_OK;
+}
+
+/* The same sums in float arithmetic, in the same order: the selection decision
+ * taken in the precision of the GPU's fp32 scores. */
+int oracle_pool_sums_f32(const float *S, int64_t n, int32_t w, float *out) {
+    if (n < 0 || w < 0) return ORACLE_EINVAL;
+    const int64_t h = w > 1 ? w / 2 : 0;
+    for (int64_t j = 0; j < n; ++j) {
+        float s = 0.0f;
+        for (int64_t k = (j - h < 0 ? 0 : j - h); k <= j + h && k < n; ++k) s += S[k];
+        out[j] = s;
+    }
     return ORACLE_OK;
 }
 

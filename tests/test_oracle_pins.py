@@ -306,3 +306,120 @@ def test_validation_rejects_bad_splits():
     p = problem(w)
     p.Hq = 5
     assert not oracle.validate(p)
+
+
+# ---------------------------------------------------------------- selection variants
+
+def row_softmax_scores(Q, K, w, u, g, norm_over_all):
+    """Library reference for the scores of chunk u: torch fp64 softmax of each
+    query row over the chunk, or over every key the row attends ([0, t]),
+    summed over the query rows and the query heads of KV head g."""
+    G = w.Hq // w.Hkv
+    off = chunk_offsets(w)
+    j0, j1 = int(off[u]), int(off[u + 1])
+    S = torch.zeros(j1 - j0, dtype=torch.float64)
+    for h in range(g * G, (g + 1) * G):
+        for i in range(w.q):
+            t = w.N - w.q + i
+            q = Q[t, h].double()
+            k0, k1 = (0, t + 1) if norm_over_all else (j0, j1)
+            x = (K[k0:k1, g].double() @ q) / math.sqrt(w.d)
+            p = torch.softmax(x, dim=0)
+            S += p[j0 - k0:j1 - k0]
+    return S.numpy()
+
+
+@pytest.mark.parametrize("norm", [0, 1])
+def test_scores_against_library_softmax(norm):
+    """Both normalisations against torch's softmax, row by row."""
+    w = small(H=2, N=260, a=12, q=6, l=8, Hq=4, Hkv=2, d=16)
+    Q, K, V, Qb, Kb, Vb = bits(w)
+    p = problem(w)
+    p.score_norm = norm
+    for u in range(2 * w.H - 1):
+        for g in range(w.Hkv):
+            np.testing.assert_allclose(oracle.chunk_scores(p, Qb, Kb, u, g),
+                                       row_softmax_scores(Q, K, w, u, g, norm == 1), rtol=1e-12, atol=1e-15)
+
+
+def test_row_normalised_scores_of_identical_keys():
+    """score_norm 1 with every key equal: each query row spreads 1/(t+1) over
+    its t+1 keys, so every key of every chunk scores sum_{h in g, i} 1/(t_i+1)."""
+    w = small(H=2, N=300, a=10, q=8, l=4)
+    Q, K, V, Qb, Kb, Vb = bits(w)
+    Kb = np.ascontiguousarray(np.broadcast_to(Kb[:1], Kb.shape))
+    p = problem(w)
+    p.score_norm = 1
+    G = w.Hq // w.Hkv
+    want = G * sum(1.0 / (w.N - w.q + i + 1) for i in range(w.q))
+    for u in range(2 * w.H - 1):
+        np.testing.assert_allclose(oracle.chunk_scores(p, Qb, Kb, u, 0), want, rtol=1e-12)
+
+
+def test_row_normalised_scores_sum_to_the_context_mass():
+    """score_norm 1: the scores of all producing chunks add up to each row's
+    attention mass on those chunks -- G*q minus the mass on the anchor, the
+    last chunk and the query block, computed here with torch."""
+    w = small(H=2, N=240, a=10, q=6, l=4, d=16)
+    Q, K, V, Qb, Kb, Vb = bits(w)
+    p = problem(w)
+    p.score_norm = 1
+    off = chunk_offsets(w)
+    G = w.Hq // w.Hkv
+    for g in range(w.Hkv):
+        total = sum(oracle.chunk_scores(p, Qb, Kb, u, g).sum() for u in range(2 * w.H - 1))
+        mass = 0.0
+        for h in range(g * G, (g + 1) * G):
+            for i in range(w.q):
+                t = w.N - w.q + i
+                x = (K[:t + 1, g].double() @ Q[t, h].double()) / math.sqrt(w.d)
+                pr = torch.softmax(x, dim=0)
+                mass += float(pr[int(off[0]):int(off[2 * w.H - 1])].sum())
+        np.testing.assert_allclose(total, mass, rtol=1e-12)
+
+
+def test_pool_sums_brute_force():
+    """Window sums against numpy's convolution with a box of w ones (zero
+    outside), float64 and float32, and w <= 1 as the identity."""
+    rng = np.random.default_rng(3)
+    for n in (1, 2, 5, 37):
+        S = rng.random(n)
+        for wdw in (1, 3, 5, 7):
+            want = np.convolve(S, np.ones(wdw), mode="same") if wdw <= n else None
+            got = oracle.pool_sums(S, wdw)
+            if want is not None:
+                np.testing.assert_allclose(got, want, rtol=1e-13)
+            # clipped window, summed directly
+            h = wdw // 2
+            direct = np.array([S[max(0, j - h):j + h + 1].sum() for j in range(n)])
+            np.testing.assert_allclose(got, direct, rtol=1e-13)
+            got32 = oracle.pool_sums(S.astype(np.float32), wdw)
+            ref32 = np.zeros(n, dtype=np.float32)
+            for j in range(n):
+                acc = np.float32(0)
+                for k in range(max(0, j - h), min(n, j + h + 1)):
+                    acc = np.float32(acc + np.float32(S[k]))
+                ref32[j] = acc
+            assert np.array_equal(got32, ref32)
+    np.testing.assert_array_equal(oracle.pool_sums(np.arange(4.0), 1), np.arange(4.0))
+
+
+def test_pooled_selection_takes_the_window_of_a_spike():
+    """One dominant score: with pooling of width w and l = w the passing block
+    is exactly the w keys centred on it (a plausible off-by-one in the window
+    fails this)."""
+    n, spike, wdw = 40, 17, 5
+    S = np.full(n, 1e-3)
+    S[spike] = 10.0
+    idx = oracle.select_top_l(oracle.pool_sums(S, wdw), 100, wdw)
+    np.testing.assert_array_equal(idx, 100 + np.arange(spike - 2, spike + 3))
+
+
+def test_variant_flags_are_validated():
+    w = small()
+    Q, K, V, Qb, Kb, Vb = bits(w)
+    for norm, pool in ((2, 0), (0, 4), (-1, 0), (0, -3)):
+        p = problem(w)
+        p.score_norm, p.score_pool = norm, pool
+        with pytest.raises(ValueError):
+            oracle.chunk_scores(p, Qb, Kb, 0, 0)
