@@ -17,6 +17,7 @@ the same workload instead (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -185,7 +186,8 @@ def oracle_sample(w, budget_s: float, inputs, seed: int = 0):
     Qb, Kb, Vb = inputs
     off = chunk_offsets(w)
     p = oracle.Problem(H=w.H, Hq=w.Hq, Hkv=w.Hkv, d=w.d, N=w.N, a=w.a, q=w.q, offsets=off,
-                       l=w.l, local_pair_full=w.local_pair_full)
+                       l=w.l, local_pair_full=w.local_pair_full, score_norm=w.score_norm,
+                       score_pool=w.score_pool)
     G = w.Hq // w.Hkv
     # (1) scores of chunk 0, KV head 0, and their selection
     t0 = time.perf_counter()
@@ -224,10 +226,16 @@ def oracle_sample(w, budget_s: float, inputs, seed: int = 0):
     return w.N / t_layer, desc, oracle.num_threads(), t_score + t_select + t_attn
 
 
+def selected_workload(args):
+    """The named layer, with the selection variant asked for (default: none)."""
+    return dataclasses.replace(WORKLOADS[args.workload], score_norm=args.score_norm,
+                               score_pool=args.score_pool)
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = selected_workload(args)
     values, cores, desc, spent = [], None, None, 0.0
     per_step = max(3.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     inputs = oracle_inputs(w)
@@ -255,7 +263,8 @@ def workload_config(w):
                         f"d={w.d}, {w.N} tokens (anchor {w.a}, query block {w.q}), top-l={w.l}",
             "tokens": w.N, "H": w.H, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
             "anchor": w.a, "query_block": w.q, "top_l": w.l,
-            "local_pair_full": w.local_pair_full,
+            "local_pair_full": w.local_pair_full, "score_norm": w.score_norm,
+            "score_pool": w.score_pool,
             "inputs": "seeded synthetic video-shaped bf16 (frame-correlated keys"
                       + (", 5% heavy-hitter keys" if w.heavy_frac else "")
                       + (", +/-10% uneven chunks" if w.jitter else "") + ")",
@@ -266,7 +275,7 @@ def workload_config(w):
 def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    w = WORKLOADS[args.workload]
+    w = selected_workload(args)
     Q, K, V, off = make_inputs(w, device)
     lay = Layout.from_workload(w)
     sp = Spava(lay, device)
@@ -395,6 +404,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--score-norm", type=int, default=0, choices=[0, 1],
+                    help="selection variant: 1 = row-normalised scores")
+    ap.add_argument("--score-pool", type=int, default=0,
+                    help="selection variant: odd window w >= 3 = pooled ranking")
     args = ap.parse_args()
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

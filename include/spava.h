@@ -74,6 +74,16 @@ typedef struct {
                                 partner chunk in full and takes no passing block from
                                 it; 0: every virtual host takes the passing blocks of
                                 all earlier chunks and no full partner chunk */
+    /* Selection variants (ablations of the score reading; the pages fix
+     * neither): */
+    int32_t score_norm;   /* 0 (default): each query row's softmax over the chunk
+                             being scored; 1: the row's own attention weights,
+                             normalised over every key it attends, [0, t] */
+    int32_t score_pool;   /* 0 or 1 (default): rank the scores themselves; odd w
+                             in 3..255: rank each key by the sum of the scores of
+                             the w keys centred on it inside its chunk (the w-key
+                             window mean with zero padding, up to the factor 1/w);
+                             spava_score still returns the unpooled scores */
 } spava_config;
 
 /* Workspace bytes that any entry point below needs for this config (the

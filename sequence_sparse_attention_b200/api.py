@@ -31,6 +31,8 @@ class Layout:
     l: int
     scale: float = 0.0
     local_pair_full: int = 1
+    score_norm: int = 0
+    score_pool: int = 0
     _keep: list = field(default_factory=list, repr=False)
 
     @classmethod
@@ -38,14 +40,15 @@ class Layout:
         from .synth import chunk_offsets
         off = chunk_offsets(w) if offsets is None else offsets
         return cls(w.H, w.Hq, w.Hkv, w.d, w.N, w.a, w.q, np.asarray(off, dtype=np.int64), w.l,
-                   0.0, w.local_pair_full)
+                   0.0, w.local_pair_full, w.score_norm, w.score_pool)
 
     def c(self) -> SpavaConfig:
         off = np.ascontiguousarray(self.offsets, dtype=np.int64)
         self._keep = [off]
         return SpavaConfig(self.H, self.Hq, self.Hkv, self.d, self.N, self.a, self.q,
                            off.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), self.l,
-                           float(self.scale), int(self.local_pair_full))
+                           float(self.scale), int(self.local_pair_full), int(self.score_norm),
+                           int(self.score_pool))
 
     @property
     def n_chunks(self) -> int:

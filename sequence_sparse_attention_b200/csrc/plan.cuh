@@ -33,11 +33,13 @@ constexpr int kMaxGroups = 2 * kMaxChunks + 8 + 2 * kMaxChunks;
 constexpr int kRowTile = 128;    // query rows per work item
 constexpr int kKeyTile = 128;    // keys per pipeline step
 constexpr int kMaxSegs = 4;      // key segments of one work item
+constexpr int kMaxPool = 255;    // widest score-pooling window
 
 enum ItemKind : int32_t { kCtx = 0, kAnchor = 1, kQueryPart = 2, kStats = 3 };
 
 struct Layer {
     int32_t H, Hq, Hkv, d, G, lpf, l, n_chunks;
+    int32_t norm, pool;                // selection variants: row-normalised scores, window width
     int32_t N, a, q, C, L;             // tokens, anchor, query, context, packed rows
     float scale_log2;                  // softmax scale * log2(e)
     int32_t off[kMaxChunks + 1];       // chunk offsets

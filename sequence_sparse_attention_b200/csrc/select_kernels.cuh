@@ -47,13 +47,27 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_sums, int *
     return before;
 }
 
-// One CTA per (chunk u < 2H-1, KV head g): the min(l, n_u) largest scores of
+// One CTA per (chunk u < 2H-1, KV head g): the min(l, n_u) largest scores (or
+// pooled window sums, rank_value) of
 // the chunk, ties to the lower token index, written ascending as absolute
 // positions; padding -1.  Radix select on the ordered 32-bit key (4 passes of
 // 8 bits) finds the exact threshold key T and how many keys equal to T are
 // kept; a final pass in index order emits the set, so the output is sorted and
 // the lower-index rule holds for the keys equal to T.
 constexpr int kSelectThreads = 1024;
+
+// The value a key is ranked by: its score, or with pooling (L.pool = w >= 3)
+// the sum of the scores of the w keys centred on it inside the chunk, added in
+// ascending order with plain fp32 adds (the window mean with zero padding up to
+// the factor 1/w, which does not change the ranking).
+__device__ __forceinline__ float rank_value(const float *S, int n, int j, int pool) {
+    if (pool <= 1) return S[j];
+    const int h = pool >> 1;
+    const int k0 = j - h < 0 ? 0 : j - h, k1 = j + h < n ? j + h : n - 1;
+    float s = 0.f;
+    for (int k = k0; k <= k1; ++k) s = __fadd_rn(s, S[k]);
+    return s;
+}
 
 __global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, const float *scores,
                                                               int32_t *idx) {
@@ -81,7 +95,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, con
         if (tid < 256) hist[tid] = 0;
         __syncthreads();
         for (int j = tid; j < n; j += blockDim.x) {
-            const uint32_t k = ordered_key(S[j]);
+            const uint32_t k = ordered_key(rank_value(S, n, j, L.pool));
             if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
         }
         __syncthreads();
@@ -110,7 +124,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, con
     const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
     int gt = 0, eq = 0;
     for (int j = j0; j < j1; ++j) {
-        const uint32_t k = ordered_key(S[j]);
+        const uint32_t k = ordered_key(rank_value(S, n, j, L.pool));
         gt += k > T;
         eq += k == T;
     }
@@ -119,7 +133,7 @@ __global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, con
     int pos = block_exclusive_scan(gt + take_eq, warp_sums, &s_total);
     int taken = 0;
     for (int j = j0; j < j1; ++j) {
-        const uint32_t k = ordered_key(S[j]);
+        const uint32_t k = ordered_key(rank_value(S, n, j, L.pool));
         if (k > T || (k == T && taken < take_eq)) {
             out[pos++] = base + j;
             taken += (k == T);

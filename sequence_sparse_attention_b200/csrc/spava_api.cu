@@ -49,6 +49,9 @@ spava_status make_layer(const spava_config *c, Layer *L) {
     if (c->anchor_len < 0 || c->query_len < 1 || c->top_l < 0 || c->n_tokens < 1)
         return SPAVA_ERR_INVALID_ARG;
     if (c->local_pair_full != 0 && c->local_pair_full != 1) return SPAVA_ERR_INVALID_ARG;
+    if (c->score_norm != 0 && c->score_norm != 1) return SPAVA_ERR_INVALID_ARG;
+    if (c->score_pool < 0 || (c->score_pool > 1 && c->score_pool % 2 == 0)) return SPAVA_ERR_INVALID_ARG;
+    if (c->score_pool > kMaxPool) return SPAVA_ERR_UNSUPPORTED;
     if (c->H > kMaxChunks / 2) return SPAVA_ERR_UNSUPPORTED;
     if (c->head_dim != 64 && c->head_dim != 128) return SPAVA_ERR_UNSUPPORTED;
     if (c->n_tokens >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
@@ -64,6 +67,8 @@ spava_status make_layer(const spava_config *c, Layer *L) {
     L->d = c->head_dim;
     L->G = c->n_q_heads / c->n_kv_heads;
     L->lpf = c->local_pair_full;
+    L->norm = c->score_norm;
+    L->pool = c->score_pool > 1 ? c->score_pool : 1;
     L->l = c->top_l;
     L->n_chunks = nc;
     L->N = static_cast<int32_t>(c->n_tokens);
@@ -118,8 +123,13 @@ int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int r
         gs.push_back({Group{kind, sub, n_rt, 0}, item_tiles(L, it)});
     };
     const int n_qrt = cdiv(L.q, kRowTile);
-    if (stats) {
+    if (stats && L.norm == 0) {
         for (int u = 0; u < L.n_chunks - 1; ++u) push(kStats, u, n_qrt);
+    } else if (stats) {
+        // Row-normalised scores: the query rows' statistics over every segment
+        // they attend (anchor, each chunk, the query block up to the row), the
+        // same segments as the query-row partials of the attention.
+        for (int s = (L.a > 0 ? 0 : 1); s < L.n_chunks + 2; ++s) push(kQueryPart, s, n_qrt);
     } else {
         for (int v = 0; v < L.n_chunks; ++v) push(kCtx, v, cdiv(L.off[v + 1] - L.off[v], kRowTile));
         if (L.a > 0) push(kAnchor, 0, cdiv(L.a, kRowTile));
@@ -272,6 +282,11 @@ spava_status launch_attn(AttnParams &p, cudaStream_t st) {
     return launched();
 }
 
+// The normaliser of the scores: per (chunk u, query head, query row) the base-2
+// log-sum-exp of the row's logits over chunk u (score_norm 0), or over every
+// key the row attends, the same value for every u (score_norm 1: the segment
+// statistics go to the query-partial lse array, free until the attention, and
+// are combined there).
 spava_status run_stats(const Layer &L, const void *q, const void *k, char *ws, cudaStream_t st) {
     const WsLayout w = ws_layout(L);
     AttnParams p;
@@ -280,9 +295,14 @@ spava_status run_stats(const Layer &L, const void *q, const void *k, char *ws, c
     SPAVA_TRY(map_tokens(&p.tmQ, q, L, L.Hq));
     SPAVA_TRY(map_tokens(&p.tmK, k, L, L.Hkv));
     p.n_groups = plan_attention(L, true, p.groups);
-    p.stats = reinterpret_cast<float *>(ws + w.stats);
+    float *stats = reinterpret_cast<float *>(ws + w.stats);
+    p.stats = L.norm ? reinterpret_cast<float *>(ws + w.part_lse) : stats;
     p.status = reinterpret_cast<int *>(ws + w.status);
-    return L.d == 128 ? launch_attn<128, true>(p, st) : launch_attn<64, true>(p, st);
+    SPAVA_TRY(L.d == 128 ? launch_attn<128, true>(p, st) : launch_attn<64, true>(p, st));
+    if (!L.norm) return SPAVA_OK;
+    const int rows = L.Hq * L.q;
+    row_lse_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, st>>>(L, p.stats, stats);
+    return launched();
 }
 
 spava_status run_scores(const Layer &L, const void *q, const void *k, float *scores, char *ws,
@@ -317,7 +337,7 @@ spava_status run_scores(const Layer &L, const void *q, const void *k, float *sco
 spava_status run_topk(const Layer &L, const float *scores, int32_t *idx, cudaStream_t st) {
     const int blocks = (L.n_chunks - 1) * L.Hkv;
     if (blocks == 0 || L.l == 0) return SPAVA_OK;
-    topk_kernel<<<blocks, kSelectThreads, 0, st>>>(L, scores, idx);
+    topk_kernel<<<blocks, kSelectThreads, 0, st>>>(L, scores, idx);  // pools on the fly (L.pool)
     return launched();
 }
 
@@ -733,6 +753,9 @@ extern "C" spava_status spava_score_noalloc(const spava_config *cfg, const void 
     SPAVA_TRY(check_ptr(q));
     SPAVA_TRY(check_ptr(k));
     SPAVA_TRY(check_ptr(scores));
+    // The fixed scratch holds the per-chunk statistics only: the row-normalised
+    // variant (statistics of every segment first) is not offered here.
+    if (L.norm) return SPAVA_ERR_UNSUPPORTED;
     const size_t stats_bytes = sizeof(float) * size_t(L.n_chunks - 1) * L.Hq * L.q;
     if (kNoAllocStatusBytes + stats_bytes > kNoAllocScratchBytes) return SPAVA_ERR_WORKSPACE;
     void *scratch = nullptr;

@@ -7,7 +7,11 @@
 // logits against each chunk u:  stats[u, h, i] = log2 sum_{j in B_u} 2^(x_ij),
 // x = scale * log2(e) * q_i . k_j  (score_kernel.cuh divides by it).
 //
-// One CTA = 128 query rows of one head against one chunk.  Warp roles:
+// With row-normalised scores the same kernel runs over every segment a query
+// row attends (anchor, chunks, the query block causally), writing one
+// statistic per segment; row_lse_kernel combines them.
+//
+// One CTA = 128 query rows of one head against one segment.  Warp roles:
 //   warps 0-7  two warps per TMEM lane quarter, each taking one half of the 128
 //              keys of a tile; running max with conditional rescaling of the
 //              running sum (the max only moves when it grows by more than 2^8)
@@ -184,7 +188,9 @@ __global__ void __launch_bounds__(kStatsThreads, 1) stats_kernel(const __grid_co
         TileCursor cur;
         for (int j = 0; j < T; ++j) {
             const Seg &s = segs[cur.seg];
-            const int lim = s.end - (s.begin + cur.tile * kKeyTile + kh * kHalf);  // valid keys
+            int lim_end = s.end;
+            if (s.causal && t + 1 < lim_end) lim_end = t + 1;  // the query block up to the row
+            const int lim = lim_end - (s.begin + cur.tile * kKeyTile + kh * kHalf);  // valid keys
             cur.advance(segs);
 
             const bool got = __all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, ab));
@@ -253,6 +259,24 @@ __global__ void __launch_bounds__(kStatsThreads, 1) stats_kernel(const __grid_co
         tc_fence_after();
         tmem_dealloc(tmem, kStatsTmemCols);
     }
+}
+
+// Row-normalised scores: the base-2 log-sum-exp of every query row over all the
+// segments it attends, seg[s][h][i] combined over s (anchor s = 0 only if
+// a > 0, chunks s = 1..2H, query block s = 2H+1), written for every producing
+// chunk u so that the scoring pass reads it like a per-chunk statistic.
+__global__ void row_lse_kernel(const Layer L, const float *seg, float *stats) {
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;  // h * q + i
+    const int rows = L.Hq * L.q;
+    if (r >= rows) return;
+    const int s0 = L.a > 0 ? 0 : 1, s1 = L.n_chunks + 1;
+    float m = -INFINITY;
+    for (int s = s0; s <= s1; ++s) m = fmaxf(m, seg[static_cast<size_t>(s) * rows + r]);
+    float sum = 0.f;
+    if (m != -INFINITY)
+        for (int s = s0; s <= s1; ++s) sum += exp2f(seg[static_cast<size_t>(s) * rows + r] - m);
+    const float lse = (m == -INFINITY) ? -INFINITY : m + log2f(sum);
+    for (int u = 0; u < L.n_chunks - 1; ++u) stats[static_cast<size_t>(u) * rows + r] = lse;
 }
 
 }  // namespace spava

@@ -37,7 +37,8 @@ class SpavaConfig(ctypes.Structure):
         ("chunk_offsets", ctypes.POINTER(ctypes.c_int64)),
         ("top_l", ctypes.c_int32),
         ("scale", ctypes.c_float),
-        ("local_pair_full", ctypes.c_int32),
+        ("local_pair_full", ctypes.c_int32), ("score_norm", ctypes.c_int32),
+        ("score_pool", ctypes.c_int32),
     ]
 
 

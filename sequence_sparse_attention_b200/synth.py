@@ -54,6 +54,8 @@ class Workload:
     jitter: float = 0.0
     seed: int = 0
     local_pair_full: int = 1
+    score_norm: int = 0     # selection variants (see spava_config)
+    score_pool: int = 0
 
     @property
     def n_chunks(self) -> int:

@@ -25,7 +25,8 @@ SCORE_REL = 1e-3
 def problem(w: Workload, off=None) -> oracle.Problem:
     return oracle.Problem(H=w.H, Hq=w.Hq, Hkv=w.Hkv, d=w.d, N=w.N, a=w.a, q=w.q,
                           offsets=chunk_offsets(w) if off is None else off, l=w.l,
-                          local_pair_full=w.local_pair_full)
+                          local_pair_full=w.local_pair_full, score_norm=w.score_norm,
+                          score_pool=w.score_pool)
 
 
 class OracleRun:
@@ -44,9 +45,11 @@ class OracleRun:
 
 
 def check_selection(w: Workload, scores_oracle: np.ndarray, idx_gpu: np.ndarray, groups):
-    """Every (chunk, group) selection is a valid top-l of the oracle scores:
-    the same set wherever the l-th / (l+1)-th gap exceeds SEL_BAND relative,
-    otherwise the same outside the band around the l-th score."""
+    """Every (chunk, group) selection is a valid top-l of the oracle scores (or
+    of their window sums, with pooling): the same set wherever the l-th /
+    (l+1)-th gap exceeds SEL_BAND relative, otherwise the same outside the band
+    around the l-th value."""
+    scores_oracle = oracle.selection_scores(problem(w), scores_oracle)
     off = chunk_offsets(w)
     n_exact = n_band = 0
     for u in range(2 * w.H - 1):

@@ -57,6 +57,10 @@ def status(fn, lay, *args):
     (dict(q=0), 1),
     (dict(l=-1), 1),
     (dict(local_pair_full=2), 1),
+    (dict(score_norm=2), 1),              # selection variants: unknown normalisation
+    (dict(score_pool=4), 1),              # even window
+    (dict(score_pool=-3), 1),
+    (dict(score_pool=257), 2),            # wider than the kernel offers
 ])
 def test_bad_config_rejected(change, expect):
     w = WORKLOADS["tiny"]
@@ -152,3 +156,16 @@ def test_zigzag_host_balance_on_equal_chunks():
     for name in ("16k", "64k", "128k"):
         _, host = attended_pairs(Layout.from_workload(WORKLOADS[name]))
         assert len(set(host)) == 1, (name, host)
+
+
+def test_variant_configs_accepted_and_noalloc_refuses_row_norm():
+    """The selection variants are valid configurations; the allocation-free
+    scoring entry (whose fixed scratch holds per-chunk statistics only) refuses
+    the row-normalised one before any CUDA call."""
+    w = WORKLOADS["tiny"]
+    for kw in (dict(score_norm=1), dict(score_pool=1), dict(score_pool=5), dict(score_norm=1, score_pool=255)):
+        n = ctypes.c_size_t()
+        assert status("spava_workspace_size", lay_of(w, **kw), ctypes.byref(n)) == 0
+    buf = ctypes.create_string_buffer(4096)
+    fake = (ctypes.addressof(buf) + 255) // 256 * 256
+    assert status("spava_score_noalloc", lay_of(w, score_norm=1), fake, fake, fake, None) == 2
