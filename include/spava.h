@@ -185,6 +185,19 @@ spava_status spava_selftest_wait_timeout(void *ws, size_t ws_bytes, void *stream
  * "Bilanciamento del Carico dell'Attenzione Approssimata").  Host only. */
 spava_status spava_attended_pairs(const spava_config *cfg, int64_t pairs[3], int64_t *per_host);
 
+/* Chunk offsets from a frame list ("Riepilogo Tecnico: APB-V", Metodologia,
+ * "Bilanciamento del Carico Visivo": the frames are spread evenly over the
+ * virtual hosts).  frame_tokens: HOST array of the n_frames frames' token
+ * counts, in order (each >= 1); the 2H chunks take consecutive whole frames,
+ * chunk v taking floor(n_frames / 2H) frames plus one more for
+ * v < n_frames mod 2H.  Writes chunk_offsets[0..2H] (HOST, int64):
+ * off[0] = anchor_len, off[v+1] = off[v] + the tokens of chunk v's frames, so a
+ * layer built from them has N = off[2H] + query_len.  SPAVA_ERR_INVALID_ARG if
+ * H is outside 1..32, n_frames < 2H (a chunk would be empty), a frame has no
+ * token, anchor_len < 0, a pointer is NULL or the sum passes 2^31.  Host only. */
+spava_status spava_plan_chunks(int32_t H, const int64_t *frame_tokens, int64_t n_frames,
+                               int64_t anchor_len, int64_t *chunk_offsets);
+
 /* spava_score for callers that cannot allocate device memory: same inputs,
  * same scores output, no workspace argument.  (The pages have no counterpart:
  * this is an interface choice of the library, not part of the method.)

@@ -99,6 +99,17 @@ def attended_pairs(lay: Layout):
     return tuple(pairs), list(per_host)
 
 
+def plan_chunks(H: int, frame_tokens, anchor_len: int) -> np.ndarray:
+    """Chunk offsets [2H+1] spreading the frames evenly over the 2H virtual
+    hosts (whole frames, consecutive, counts differing by at most one)."""
+    ft = np.ascontiguousarray(frame_tokens, dtype=np.int64)
+    off = np.empty(2 * H + 1, dtype=np.int64)
+    P = ctypes.POINTER(ctypes.c_int64)
+    native.call("spava_plan_chunks", int(H), ft.ctypes.data_as(P), len(ft), int(anchor_len),
+                off.ctypes.data_as(P))
+    return off
+
+
 def new_workspace(lay: Layout, device) -> torch.Tensor:
     """A zeroed workspace (the status word must start at zero)."""
     return torch.zeros(workspace_size(lay), dtype=torch.uint8, device=device)

@@ -658,6 +658,27 @@ spava_status spava_selftest_wait_timeout(void *ws, size_t ws_bytes, void *stream
     return launched();
 }
 
+spava_status spava_plan_chunks(int32_t H, const int64_t *frame_tokens, int64_t n_frames,
+                               int64_t anchor_len, int64_t *chunk_offsets) {
+    if (!frame_tokens || !chunk_offsets || H < 1 || H > kMaxChunks / 2 || anchor_len < 0)
+        return SPAVA_ERR_INVALID_ARG;
+    const int nc = 2 * H;
+    if (n_frames < nc) return SPAVA_ERR_INVALID_ARG;
+    const int64_t per = n_frames / nc, extra = n_frames % nc;
+    int64_t f = 0, tok = anchor_len;
+    chunk_offsets[0] = anchor_len;
+    for (int v = 0; v < nc; ++v) {
+        const int64_t take = per + (v < extra ? 1 : 0);
+        for (int64_t i = 0; i < take; ++i, ++f) {
+            if (frame_tokens[f] < 1) return SPAVA_ERR_INVALID_ARG;
+            tok += frame_tokens[f];
+            if (tok >= (1LL << 31)) return SPAVA_ERR_INVALID_ARG;
+        }
+        chunk_offsets[v + 1] = tok;
+    }
+    return SPAVA_OK;
+}
+
 spava_status spava_attended_pairs(const spava_config *cfg, int64_t pairs[3], int64_t *per_host) {
     Layer L;
     SPAVA_TRY(make_layer(cfg, &L));

@@ -169,3 +169,44 @@ def test_variant_configs_accepted_and_noalloc_refuses_row_norm():
     buf = ctypes.create_string_buffer(4096)
     fake = (ctypes.addressof(buf) + 255) // 256 * 256
     assert status("spava_score_noalloc", lay_of(w, score_norm=1), fake, fake, fake, None) == 2
+
+
+def test_plan_chunks_spreads_frames_evenly():
+    """Visual load balancing: consecutive whole frames, counts differing by at
+    most one with the extra frames in the first chunks; offsets accumulate the
+    frames' tokens from the anchor on, and form a valid layer."""
+    from sequence_sparse_attention_b200.api import plan_chunks
+    rng = np.random.default_rng(5)
+    for H, n_frames in ((1, 2), (2, 9), (4, 64), (8, 1006), (3, 37)):
+        ft = rng.integers(100, 300, n_frames)
+        off = plan_chunks(H, ft, 64)
+        nc = 2 * H
+        counts = [n_frames // nc + (1 if v < n_frames % nc else 0) for v in range(nc)]
+        bounds = np.concatenate([[0], np.cumsum(counts)])
+        want = 64 + np.concatenate([[0], np.cumsum(ft)])[bounds]
+        np.testing.assert_array_equal(off, want)
+        lay = Layout(H, 4, 2, 64, int(off[-1]) + 16, 64, 16, off, 8)
+        n = ctypes.c_size_t()
+        assert status("spava_workspace_size", lay, ctypes.byref(n)) == 0
+
+
+def test_plan_chunks_equal_frames_divide_evenly():
+    """Equal frames whose count divides by 2H: every chunk gets the same number
+    of whole frames."""
+    from sequence_sparse_attention_b200.api import plan_chunks
+    off = plan_chunks(4, [256] * 64, 1024)
+    np.testing.assert_array_equal(off, 1024 + 256 * 8 * np.arange(9))
+
+
+@pytest.mark.parametrize("args", [
+    (0, [5, 5], 0), (33, [1] * 66, 0),    # H out of range
+    (2, [5, 5, 5], 0),                    # fewer frames than chunks
+    (1, [5, 0], 0),                       # a frame without tokens
+    (1, [5, 5], -1),                      # negative anchor
+    (1, [2 ** 30, 2 ** 30], 0),           # past 2^31 tokens
+])
+def test_plan_chunks_rejects(args):
+    from sequence_sparse_attention_b200.api import plan_chunks
+    from sequence_sparse_attention_b200.native import SpavaError
+    with pytest.raises(SpavaError):
+        plan_chunks(*args)
