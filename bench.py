@@ -341,6 +341,28 @@ def run_ours(args, world, rank, local):
                 "frac_of_burst_peak": achieved / pk_.get("bf16_tflops", peak),
                 "algorithmic_flops_per_launch": flops, "attended_pairs_per_head": pairs}
 
+    # ---- the selection phase against HBM (each operand touched once)
+    hbm = pk_.get("hbm_gbs")
+    n_sel = sum(min(w.l, int(off[u + 1] - off[u])) for u in range(2 * w.H - 1))
+    packed_rows = w.Hkv * (w.a + n_sel)
+    scored = int(off[2 * w.H - 1]) - w.a    # keys of the producing chunks
+    sel_bytes = {
+        # K of the scored chunks read twice (statistics, scores), the query
+        # block's Q rows, the scores written
+        "score": 2 * scored * w.Hkv * w.d * 2 + w.q * w.Hq * w.d * 2 + 4 * w.Hkv * scored,
+        # scores read, indices written
+        "topk": 4 * w.Hkv * scored + 4 * (2 * w.H - 1) * w.Hkv * w.l,
+        # K and V rows read and written
+        "pack": 2 * 2 * packed_rows * w.d * 2,
+    }
+    selection = {k: {"bytes": b, "GB/s": b / (per[k] / 1e3) / 1e9,
+                     "frac_of_hbm": b / (per[k] / 1e3) / 1e9 / hbm}
+                 for k, b in sel_bytes.items()}
+    selection["peak_GBps"] = hbm
+    selection["note"] = ("pack (the gather) is the HBM-bound step; scoring is tensor/exp-bound "
+                         "(one exponential per 4*d flops) and top-l latency-bound, so their GB/s "
+                         "fractions are reported, not targeted")
+
     # ---- end to end through the host-buffer entry point
     qh = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
     kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
@@ -381,6 +403,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": workload_config(w),
         "roofline": roofline,
+        "selection_hbm": selection,
         "kernel_ms": per,
         "tensor_peak_frac": {"of_sustained": achieved / peak,
                              "of_burst": achieved / pk_.get("bf16_tflops", peak),
