@@ -91,23 +91,44 @@ static_assert(128 * kRegsIo + 256 * kRegsSoftmax <= kAttnThreads * kLaunchRegs,
 constexpr int kColO = 256;  // O_A; O_B at kColO + 128
 constexpr int kItemBar = 1;  // named barrier of all threads between work items
 
-// Work item = row tiles 2p and 2p+1 of a region.  Inside a group: KV head by KV
-// head, pairs in descending cost, the query heads of a KV head adjacent.
-__host__ __device__ inline int pair_count(int n_rt) { return (n_rt + 1) / 2; }
+// Work items of a region (one group): row tiles 2p and 2p+1 of one query head;
+// when the region has an odd number of row tiles, its last tile (the costliest,
+// alone) is paired ACROSS query heads instead -- heads 2k and 2k+1 of a KV head
+// share that tile's rows, key sequence and K/V, and differ only in Q -- so that
+// at most one tile per KV head runs alone.  Inside a group: KV head by KV head,
+// the cross-head items first (costliest), then the row pairs in descending
+// cost, the query heads of a KV head adjacent.
+__host__ __device__ inline int pair_items(int n_rt, int G) {
+    return (n_rt / 2) * G + ((n_rt & 1) ? (G + 1) / 2 : 0);
+}
 
-__host__ __device__ inline Item decode_pair_item(const Group *groups, int n_groups, int b, int G) {
+// Item b: tile A = row tile it.rt of head it.h; tile B = row tile it.rt + 1 of
+// the same head (*h_b = it.h), or the same row tile of head *h_b = it.h + 1
+// (cross-head item), or none (*h_b = -1).
+__host__ __device__ inline Item decode_pair_item(const Group *groups, int n_groups, int b, int G,
+                                                 int *h_b) {
     int k = 0;
     while (k + 1 < n_groups && b >= groups[k + 1].item_begin) ++k;
     const Group &g = groups[k];
     const int i = b - g.item_begin;
-    const int np = pair_count(g.n_rt);
-    const int per_kv = np * G;
-    const int rem = i % per_kv;
+    const int per_kv = pair_items(g.n_rt, G);
+    const int kv = i / per_kv;
+    int rem = i % per_kv;
     Item it;
     it.kind = g.kind;
     it.sub = g.sub;
+    const int n_cross = (g.n_rt & 1) ? (G + 1) / 2 : 0;
+    if (rem < n_cross) {
+        it.rt = g.n_rt - 1;
+        it.h = kv * G + 2 * rem;
+        *h_b = (2 * rem + 1 < G) ? it.h + 1 : -1;
+        return it;
+    }
+    rem -= n_cross;
+    const int np = g.n_rt / 2;
     it.rt = 2 * (np - 1 - rem / G);  // first row tile of the pair
-    it.h = (i / per_kv) * G + rem % G;
+    it.h = kv * G + rem % G;
+    *h_b = it.h;
     return it;
 }
 
@@ -129,6 +150,7 @@ __device__ __forceinline__ float max128(const float (&x)[128]) {
 // key segments and tile counts.
 struct ItemPlan {
     Item it;
+    int hB;  // query head of tile B
     int r0A, eA, r0B, eB;
     bool hasB;
     Seg segs[kMaxSegs];
@@ -137,19 +159,32 @@ struct ItemPlan {
 
 __device__ __forceinline__ void plan_item(const Layer &L, const Group *groups, int n_groups, int b,
                                           ItemPlan &ip) {
-    ip.it = decode_pair_item(groups, n_groups, b, L.G);
+    int h_b;
+    ip.it = decode_pair_item(groups, n_groups, b, L.G, &h_b);
+    item_rows(L, ip.it, ip.r0A, ip.eA);
+    ip.g = ip.it.h / L.G;
+    if (h_b != ip.it.h) {
+        // Cross-head item (or a tile alone): B has A's rows and key sequence.
+        ip.hasB = h_b >= 0;
+        ip.hB = h_b;
+        ip.r0B = ip.r0A, ip.eB = ip.eA;
+        ip.ns = build_segments(L, ip.it, ip.segs);
+        ip.T = count_tiles(ip.segs, ip.ns);
+        ip.TA = ip.T;
+        ip.TB = ip.hasB ? ip.T : 0;
+        return;
+    }
     Item it_b = ip.it;
     it_b.rt = ip.it.rt + 1;
-    item_rows(L, ip.it, ip.r0A, ip.eA);
     item_rows(L, it_b, ip.r0B, ip.eB);
     ip.hasB = ip.eB > ip.r0B;
+    ip.hB = ip.it.h;
     ip.ns = build_segments(L, ip.hasB ? it_b : ip.it, ip.segs);
     ip.T = count_tiles(ip.segs, ip.ns);
     // A causal last segment starts on a tile boundary of the region, so its last
     // tile for B is B's diagonal, which lies beyond every row of A.
     ip.TA = (ip.hasB && ip.ns > 0 && ip.segs[ip.ns - 1].causal) ? ip.T - 1 : ip.T;
     ip.TB = ip.hasB ? ip.T : 0;
-    ip.g = ip.it.h / L.G;
 }
 
 template <int D>
@@ -261,7 +296,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 tma_load_3d(smem + SM::kOffQ + p * 16384, &P.tmQ, p * 64, it.h, r0A, q_full);
             if (hasB)
                 for (int p = 0; p < SM::kPanels; ++p)
-                    tma_load_3d(smem + SM::kOffQ + SM::kTile + p * 16384, &P.tmQ, p * 64, it.h, r0B,
+                    tma_load_3d(smem + SM::kOffQ + SM::kTile + p * 16384, &P.tmQ, p * 64, ip.hB, r0B,
                                 q_full);
             int k_last[KS], v_last[VS];
             for (int i = 0; i < KS; ++i) k_last[i] = -1;
@@ -408,6 +443,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         const Seg *segs = ip.segs;
         // ------------------------------------------------------------ softmax
         const int x = warp >> 2, quarter = warp & 3;
+        const int hx = x ? ip.hB : it.h;  // query head of this warp's tile
         const int TX = x ? TB : TA;
         const int row0 = x ? r0B : r0A, row_end = x ? eB : eA;
         const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
@@ -507,7 +543,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 const float lse2 = (l_run > 0.f) ? m_run + __log2f(l_run) : -INFINITY;
                 if (it.kind == kQueryPart) {
                     const int i = t - (L.N - L.q);
-                    float *dst = P.part_O + ((static_cast<size_t>(it.sub) * L.Hq + it.h) * L.q + i) * D;
+                    float *dst = P.part_O + ((static_cast<size_t>(it.sub) * L.Hq + hx) * L.q + i) * D;
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t u[32];
@@ -522,9 +558,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                                                 __uint_as_float(u[e + 2]) * inv, __uint_as_float(u[e + 3]) * inv);
                         }
                     }
-                    if (valid) P.part_lse[(static_cast<size_t>(it.sub) * L.Hq + it.h) * L.q + i] = lse2;
+                    if (valid) P.part_lse[(static_cast<size_t>(it.sub) * L.Hq + hx) * L.q + i] = lse2;
                 } else {
-                    __nv_bfloat16 *dst = P.O + (static_cast<size_t>(t) * L.Hq + it.h) * D;
+                    __nv_bfloat16 *dst = P.O + (static_cast<size_t>(t) * L.Hq + hx) * D;
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t u[32];
@@ -543,7 +579,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                             }
                         }
                     }
-                    if (valid && P.lse) P.lse[static_cast<size_t>(it.h) * L.N + t] = lse2 * 0.69314718055994531f;
+                    if (valid && P.lse) P.lse[static_cast<size_t>(hx) * L.N + t] = lse2 * 0.69314718055994531f;
                 }
             }
         }

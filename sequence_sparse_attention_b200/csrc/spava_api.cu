@@ -140,16 +140,16 @@ int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int r
     int begin = 0, n = 0;
     for (auto &g : gs) {
         g.g.item_begin = begin;
-        begin += (stats ? g.g.n_rt : pair_count(g.g.n_rt)) * L.Hq;
+        begin += stats ? g.g.n_rt * L.Hq : pair_items(g.g.n_rt, L.G) * L.Hkv;
         out[n++] = g.g;
     }
     return n;
 }
 
-int64_t plan_items(const Group *g, int n, int Hq, bool stats) {
+int64_t plan_items(const Group *g, int n, const Layer &L, bool stats) {
     if (!n) return 0;
-    const int per = stats ? g[n - 1].n_rt : pair_count(g[n - 1].n_rt);
-    return static_cast<int64_t>(g[n - 1].item_begin) + static_cast<int64_t>(per) * Hq;
+    const int per = stats ? g[n - 1].n_rt * L.Hq : pair_items(g[n - 1].n_rt, L.G) * L.Hkv;
+    return static_cast<int64_t>(g[n - 1].item_begin) + per;
 }
 
 // ---------------------------------------------------------------- workspace
@@ -254,7 +254,7 @@ spava_status launched() {
 // ---------------------------------------------------------------- launches
 template <int D, bool STATS>
 spava_status launch_attn(AttnParams &p, cudaStream_t st) {
-    const int64_t items = plan_items(p.groups, p.n_groups, p.L.Hq, STATS);
+    const int64_t items = plan_items(p.groups, p.n_groups, p.L, STATS);
     if (items == 0) return SPAVA_OK;
     if (items >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
     if (STATS) {
