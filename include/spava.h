@@ -88,7 +88,11 @@ typedef struct {
 
 /* Workspace bytes that any entry point below needs for this config (the
  * largest of them: spava_prefill_attention).  Pass the same buffer to every
- * call; it must be 256-byte aligned. */
+ * call; it must be 256-byte aligned.  Its first 256 bytes are the status block:
+ * the status word at byte 0 (must start at zero; see spava_device_status) and
+ * the work-item counter of the attention kernel's persistent grid at byte 128
+ * (zeroed by every spava_attn before its launch).  Calls that share a
+ * workspace must be ordered on one stream. */
 spava_status spava_workspace_size(const spava_config *cfg, size_t *bytes);
 
 /* L = a + sum_u min(l, n_u): rows of the packed passing K/V per KV head. */
@@ -98,17 +102,20 @@ spava_status spava_packed_len(const spava_config *cfg, int64_t *rows);
  * KV head g and key j of chunk u,
  *   scores[g, j-a] = sum_{h in group g} sum_{i in query block}
  *                    softmax_{j' in chunk u}(scale * q_{h,i} . k_{g,j'}) at j'=j.
- * The softmax runs over chunk u only; no causal mask.  The last chunk has no
- * successor and its columns are left untouched.  Two passes over K: row
- * statistics, then probability column sums.  Reads q, k; writes scores. */
+ * The softmax runs over chunk u only (score_norm 0); no causal mask.  With
+ * score_norm 1 each row's weights are instead normalised over every key the
+ * row attends, [0, t].  The last chunk has no successor and its columns are
+ * left untouched.  Two passes over K: row statistics, then probability column
+ * sums.  Reads q, k; writes scores. */
 spava_status spava_score(const spava_config *cfg, const void *q, const void *k, float *scores,
                          void *ws, size_t ws_bytes, void *stream);
 
 /* Passing-block selection ("Blocchi di Passaggio": the most essential KV): for
  * every chunk u < 2H-1 and KV head g, the min(l, n_u) largest scores of chunk u
- * (ties: the lower token index wins), written as ascending absolute positions
- * into idx[u, g, :], the remaining slots set to -1.  Exact: no approximation
- * in the selection. */
+ * (with score_pool w >= 3: the largest sums of the w scores centred on each key
+ * inside the chunk, added in ascending order in fp32; ties: the lower token
+ * index wins), written as ascending absolute positions into idx[u, g, :], the
+ * remaining slots set to -1.  Exact: no approximation in the selection. */
 spava_status spava_topk_select(const spava_config *cfg, const float *scores, int32_t *idx,
                                void *stream);
 
