@@ -43,8 +43,8 @@ KERNELS_PER_STEP = 6   # stats, scores, top-l, pack, attention, query merge
 # DRAM traffic of one attention launch on the 128K layer, from the single-pass
 # ncu capture summarised in profiles/ (dram__bytes_read.sum + dram__bytes_write.sum);
 # valid only while the sources that decide it are unchanged (KERNEL_FILES).
-PROFILED_TRAFFIC = {"kernel_sha256": "455cfe8879c44f4c32fb09f8f2ee40d04b83e959342ba5ef4a3536baa0d34e3d",
-                    "bytes_per_launch": 3092664320 + 1211644672, "workload": "128k",
+PROFILED_TRAFFIC = {"kernel_sha256": "8f40f42cc5b61480e52ad2d2ad13b0d32e2844cbc65166ed56900f99637c762f",
+                    "bytes_per_launch": 3134094336 + 1215067648, "workload": "128k",
                     "source": "profiles/attn_kernel_128k_dram.md"}
 KERNEL_FILES = ("attn_kernel.cuh", "plan.cuh", "sm100.cuh")  # what decides the attention launch
 
