@@ -69,12 +69,12 @@ __device__ __forceinline__ float rank_value(const float *S, int n, int j, int po
     return s;
 }
 
-__global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, const float *scores,
-                                                              int32_t *idx) {
+// The selection of one (chunk u, KV head g) by the whole CTA; returns l_eff.
+__device__ __forceinline__ int select_chunk(const Layer &L, const float *scores, int32_t *idx, int u,
+                                            int g) {
     __shared__ int hist[256];
     __shared__ int warp_sums[32];
     __shared__ int s_digit, s_need, s_total;
-    const int u = blockIdx.x / L.Hkv, g = blockIdx.x % L.Hkv;
     const int base = L.off[u];
     const int n = L.off[u + 1] - base;
     const int l_eff = min(L.l, n);
@@ -83,10 +83,10 @@ __global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, con
     const int tid = threadIdx.x;
 
     for (int r = l_eff + tid; r < L.l; r += blockDim.x) out[r] = -1;
-    if (l_eff == 0) return;
+    if (l_eff == 0) return 0;
     if (l_eff == n) {
         for (int r = tid; r < n; r += blockDim.x) out[r] = base + r;
-        return;
+        return l_eff;
     }
 
     uint32_t prefix = 0, mask = 0;
@@ -138,6 +138,70 @@ __global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, con
             out[pos++] = base + j;
             taken += (k == T);
         }
+    }
+    return l_eff;
+}
+
+__global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, const float *scores,
+                                                              int32_t *idx) {
+    select_chunk(L, scores, idx, blockIdx.x / L.Hkv, blockIdx.x % L.Hkv);
+}
+
+// Copies packed rows [r0, r1) of KV head g from the token rows src(r): one warp
+// per row, lanes 0-15 the K row and lanes 16-31 the V row in 16-byte pieces,
+// 8 rows in flight per warp.
+template <int D, typename Src>
+__device__ __forceinline__ void copy_rows(const Layer &L, const __nv_bfloat16 *K,
+                                          const __nv_bfloat16 *V, __nv_bfloat16 *PK,
+                                          __nv_bfloat16 *PV, int g, int r0, int r1, int warp0,
+                                          int n_warps, Src src) {
+    constexpr int kPieces = D * 2 / 16;
+    const int lane = threadIdx.x & 31, half = lane >> 4, c = lane & 15;
+    const __nv_bfloat16 *from = half ? V : K;
+    __nv_bfloat16 *to = half ? PV : PK;
+    for (int b = r0 + warp0 * 8; b < r1; b += n_warps * 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            v[k] = make_uint4(0, 0, 0, 0);
+            if (b + k < r1 && c < kPieces) {
+                const int t = src(b + k);
+                v[k] = __ldg(reinterpret_cast<const uint4 *>(from + (static_cast<size_t>(t) * L.Hkv + g) * D) + c);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (b + k < r1 && c < kPieces)
+                reinterpret_cast<uint4 *>(to + (static_cast<size_t>(g) * L.L + b + k) * D)[c] = v[k];
+    }
+}
+
+// Selection and gather in one launch (the layer entry points): CTA (u, g) for
+// u < 2H-1 selects the passing block of chunk u for KV head g exactly as
+// topk_kernel, then copies those K/V rows to the packed rows pcum[u] + r; the
+// CTAs after them copy the anchor rows.  The selected indices are read back
+// from idx by the CTA that wrote them (visible after __syncthreads).
+constexpr int kAnchorRowsPerCta = 256;
+template <int D>
+__global__ void __launch_bounds__(kSelectThreads) select_pack_kernel(
+    const Layer L, const float *scores, int32_t *idx, const __nv_bfloat16 *K,
+    const __nv_bfloat16 *V, __nv_bfloat16 *PK, __nv_bfloat16 *PV) {
+    const int n_sel = (L.n_chunks - 1) * L.Hkv;
+    const int warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
+    if (static_cast<int>(blockIdx.x) < n_sel) {
+        const int u = blockIdx.x / L.Hkv, g = blockIdx.x % L.Hkv;
+        const int l_eff = select_chunk(L, scores, idx, u, g);
+        __syncthreads();
+        const int32_t *sel = idx + (static_cast<size_t>(u) * L.Hkv + g) * L.l;
+        const int p0 = L.pcum[u];
+        copy_rows<D>(L, K, V, PK, PV, g, p0, p0 + l_eff, warp, n_warps,
+                     [&](int r) { return sel[r - p0]; });
+    } else {
+        const int b = blockIdx.x - n_sel;
+        const int per_g = (L.a + kAnchorRowsPerCta - 1) / kAnchorRowsPerCta;
+        const int g = b / per_g, r0 = (b % per_g) * kAnchorRowsPerCta;
+        const int r1 = min(L.a, r0 + kAnchorRowsPerCta);
+        copy_rows<D>(L, K, V, PK, PV, g, r0, r1, warp, n_warps, [](int r) { return r; });
     }
 }
 

@@ -363,6 +363,24 @@ spava_status run_pack(const Layer &L, const void *k, const void *v, const int32_
     return launched();
 }
 
+// Selection and gather in one launch (select_pack_kernel): one CTA per
+// (producing chunk, KV head), then the anchor rows.
+spava_status run_select_pack(const Layer &L, const float *scores, int32_t *idx, const void *k,
+                             const void *v, void *pk, void *pv, cudaStream_t st) {
+    const int64_t n_sel = static_cast<int64_t>(L.n_chunks - 1) * L.Hkv;
+    const int64_t n_anchor = L.a > 0 ? static_cast<int64_t>(L.Hkv) * cdiv(L.a, kAnchorRowsPerCta) : 0;
+    const unsigned blocks = static_cast<unsigned>(n_sel + n_anchor);
+    auto K = static_cast<const __nv_bfloat16 *>(k);
+    auto V = static_cast<const __nv_bfloat16 *>(v);
+    auto PK = static_cast<__nv_bfloat16 *>(pk);
+    auto PV = static_cast<__nv_bfloat16 *>(pv);
+    if (L.d == 128)
+        select_pack_kernel<128><<<blocks, kSelectThreads, 0, st>>>(L, scores, idx, K, V, PK, PV);
+    else
+        select_pack_kernel<64><<<blocks, kSelectThreads, 0, st>>>(L, scores, idx, K, V, PK, PV);
+    return launched();
+}
+
 spava_status run_attn(const Layer &L, const void *q, const void *k, const void *v, const void *pk,
                       const void *pv, void *o, float *lse, char *ws, cudaStream_t st,
                       int row_lo = 0, int row_hi = INT32_MAX) {
@@ -406,10 +424,11 @@ spava_status run_front(const Layer &L, const void *q, const void *k, const void 
     if (L.n_chunks > 1 && L.l > 0) {
         SPAVA_TRY(run_stats(L, q, k, w, st));
         SPAVA_TRY(run_scores(L, q, k, scores, w, st));
-        SPAVA_TRY(run_topk(L, scores, idx, st));
+        if (v_ready) SPAVA_CUDA(cudaStreamWaitEvent(st, v_ready, 0));
+        return run_select_pack(L, scores, idx, k, v, w + lay.pk, w + lay.pv, st);
     }
     if (v_ready) SPAVA_CUDA(cudaStreamWaitEvent(st, v_ready, 0));
-    return run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st);
+    return run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st);  // anchor rows only
 }
 
 // Row groups of the copy/compute pipeline of the host entry point, in the
