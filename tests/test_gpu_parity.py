@@ -52,6 +52,13 @@ CASES = {
                        seed=23, score_pool=5),
     "rownorm_pooled": Workload("rownorm_pooled", H=2, Hq=8, Hkv=2, d=128, N=1300, a=0, q=90, l=40,
                                frame=32, seed=24, score_norm=1, score_pool=7),
+    # sixteen chunks shorter than one row tile, and the pure-virtual pairing on d = 64
+    "many_hosts": Workload("many_hosts", H=8, Hq=6, Hkv=2, d=128, N=2150, a=100, q=60, l=30,
+                           frame=16, seed=25),
+    "pure_d64": Workload("pure_d64", H=3, Hq=4, Hkv=1, d=64, N=1400, a=50, q=100, l=70, frame=32,
+                         seed=26, local_pair_full=0),
+    "variants_d64": Workload("variants_d64", H=3, Hq=6, Hkv=3, d=64, N=1500, a=64, q=140, l=50,
+                             frame=32, seed=27, score_norm=1, score_pool=3),
 }
 
 _cache = {}
@@ -190,7 +197,8 @@ def test_repeat_calls_bit_identical():
     assert torch.equal(l1, l2)
 
 
-@pytest.mark.parametrize("name", ["tiny", "g7", "no_anchor", "long_anchor", "short_chunks"])
+@pytest.mark.parametrize("name", ["tiny", "g7", "no_anchor", "long_anchor", "short_chunks",
+                                  "one_host", "many_hosts", "rownorm_pooled"])
 @pytest.mark.parametrize("pipelined", [False, True])
 def test_host_buffers_entry_point(name, pipelined):
     """Host buffers in and out, on one stream or with the copies on a second
