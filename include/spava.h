@@ -218,15 +218,23 @@ spava_status spava_plan_chunks(int32_t H, const int64_t *frame_tokens, int64_t n
  * (e.g. H=16, Hq=32, q=512 needs 2 MiB); larger layers get
  * SPAVA_ERR_WORKSPACE and nothing is launched.  No allocation of any kind
  * (no cudaMalloc, cudaFree or allocating library routine).
- * The first call on each device looks up the array's device address with
- * that device current; make that first call before any stream capture.
+ * Each call looks up the array's device address with the calling thread's
+ * current device (cudaGetSymbolAddress; the first lookup on a device loads the
+ * library's module there): make the first call on a device before any stream
+ * capture.
  * All calls share the one array: calls that overlap on the GPU (other streams,
  * other host threads) race and must be serialised by the caller.  A kernel
  * wait that gives up is recorded in the array's status word, which each call
- * clears at its start; it is not reported to the caller (use spava_score with
- * a workspace and spava_device_status where that matters). */
+ * clears at its start; read it with spava_score_noalloc_status. */
 spava_status spava_score_noalloc(const spava_config *cfg, const void *q, const void *k,
                                  float *scores, void *stream);
+
+/* Status of the last spava_score_noalloc call on the current device (the
+ * pages have no counterpart): synchronises `stream`, reads the status word of
+ * the library's fixed scratch array (bit 0: a bounded wait in a kernel gave
+ * up, the scores are incomplete), writes it to *flags and clears it.  Returns
+ * SPAVA_ERR_TIMEOUT if bit 0 was set, SPAVA_OK otherwise.  Allocates nothing. */
+spava_status spava_score_noalloc_status(void *stream, int32_t *flags);
 
 const char *spava_status_string(spava_status s);
 

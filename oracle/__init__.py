@@ -75,6 +75,8 @@ def _load():
         lib.oracle_pool_sums_f32.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_int64,
                                              ctypes.c_int32, ctypes.POINTER(ctypes.c_float)]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_attended_pairs.argtypes = [P(_Cfg), c_i64p]
+        lib.oracle_plan_chunks.argtypes = [ctypes.c_int32, c_i64p, ctypes.c_int64, ctypes.c_int64, c_i64p]
         _lib = lib
     return _lib
 
@@ -121,6 +123,20 @@ def num_threads() -> int:
 
 def pair(H: int, v: int) -> int:
     return int(_load().oracle_pair(H, v))
+
+
+def plan_chunks(H: int, frame_tokens, anchor_len: int) -> np.ndarray:
+    """Chunk offsets ``[2H+1]`` of the visual load balancing: whole,
+    consecutive frames, frame counts dealt out evenly over the 2H virtual
+    hosts (the first hosts take the extra ones)."""
+    ft = np.ascontiguousarray(frame_tokens, dtype=np.int64)
+    off = np.empty(2 * H + 1, dtype=np.int64)
+    P = ctypes.POINTER(ctypes.c_int64)
+    rc = _load().oracle_plan_chunks(int(H), ft.ctypes.data_as(P), len(ft), int(anchor_len),
+                                    off.ctypes.data_as(P))
+    if rc != 0:
+        raise ValueError(f"oracle_plan_chunks failed ({rc})")
+    return off
 
 
 def validate(p: Problem) -> bool:
@@ -217,6 +233,17 @@ def key_set(p: Problem, idx: np.ndarray, t: int, g: int) -> np.ndarray:
     if n < 0:
         raise ValueError(f"oracle_key_set failed ({n})")
     return keys[:n].copy()
+
+
+def attended_pairs(p: Problem):
+    """(anchor, context, query) attended (row, key) pairs per query head,
+    counted from the key-set definition without listing keys."""
+    cfg = p.c()
+    out = (ctypes.c_int64 * 3)()
+    rc = _load().oracle_attended_pairs(ctypes.byref(cfg), out)
+    if rc != 0:
+        raise ValueError(f"oracle_attended_pairs failed ({rc})")
+    return tuple(int(x) for x in out)
 
 
 def prefill_rows(p: Problem, Q, K, V, idx, rows, heads):

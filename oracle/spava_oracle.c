@@ -111,6 +111,38 @@ int oracle_validate(const oracle_cfg *c) {
     return ORACLE_OK;
 }
 
+/* Visual load balancing ([APB-V-IT] "Bilanciamento del Carico Visivo": the
+ * video frames are spread evenly over the virtual hosts, so that no host's
+ * share of the vision encoder is a bottleneck).  Reading: every virtual host
+ * takes whole, consecutive frames; the frames are dealt out to the 2H hosts in
+ * turn, frame f counting toward host f mod 2H, so the hosts' frame counts
+ * differ by at most one and the larger counts go to the lower hosts; host v's
+ * frames then follow those of hosts 0..v-1.  The chunk offsets are the token
+ * positions where the hosts' runs start: off[0] = a (after the anchor),
+ * off[v+1] = off[v] + the tokens of host v's frames.  n_frames >= 2H and every
+ * frame has at least one token. */
+int oracle_plan_chunks(int32_t H, const int64_t *frame_tokens, int64_t n_frames, int64_t a,
+                       int64_t *off) {
+    if (H < 1 || !frame_tokens || !off || a < 0) return ORACLE_EINVAL;
+    const int nc = 2 * H;
+    if (n_frames < nc) return ORACLE_EINVAL;
+    int64_t *count = (int64_t *)calloc((size_t)nc, sizeof(int64_t));
+    if (!count) return ORACLE_ENOMEM;
+    for (int64_t f = 0; f < n_frames; ++f) count[f % nc] += 1; /* deal the frames */
+    int64_t f = 0;
+    off[0] = a;
+    for (int v = 0; v < nc; ++v) {
+        int64_t tok = 0;
+        for (int64_t i = 0; i < count[v]; ++i, ++f) {
+            if (frame_tokens[f] < 1) { free(count); return ORACLE_EINVAL; }
+            tok += frame_tokens[f];
+        }
+        off[v + 1] = off[v] + tok;
+    }
+    free(count);
+    return ORACLE_OK;
+}
+
 /* Physical host of virtual host v under the ZigZag layout: host h holds the
  * virtual hosts h and 2H-1-h ([APB-V-IT] "Disposizione ZigZag"). */
 int oracle_pair(int H, int v) { return v < H ? v : 2 * H - 1 - v; }
@@ -283,6 +315,33 @@ int64_t oracle_key_set(const oracle_cfg *c, const int32_t *idx, int64_t t, int g
         if (take[j]) keys[n++] = j;
     free(take);
     return n;
+}
+
+/* Number of (row, key) pairs per query head that the key sets above attend,
+ * by row class (out[0] anchor rows, out[1] context rows, out[2] query rows),
+ * counted from the same definition without listing the keys: an anchor or
+ * query row t attends t+1 keys; a row at position r (0-based) of chunk v
+ * attends a + the passing-block sizes min(l, n_u) of the earlier chunks it
+ * takes + the partner chunk's n_p (v >= H, local_pair_full) + r + 1. */
+int oracle_attended_pairs(const oracle_cfg *c, int64_t *out) {
+    if (oracle_validate(c) != ORACLE_OK || !out) return ORACLE_EINVAL;
+    const int H = c->H, nc = 2 * H;
+    out[0] = c->a * (c->a + 1) / 2;
+    out[1] = 0;
+    for (int v = 0; v < nc; ++v) {
+        const int64_t n_v = c->off[v + 1] - c->off[v];
+        int64_t fixed = c->a;
+        for (int u = 0; u < v; ++u) {
+            if (c->local_pair_full && oracle_pair(H, u) == oracle_pair(H, v)) continue;
+            const int64_t n_u = c->off[u + 1] - c->off[u];
+            fixed += n_u < c->l ? n_u : c->l;
+        }
+        if (c->local_pair_full && v >= H) fixed += c->off[nc - v] - c->off[nc - 1 - v];
+        out[1] += n_v * fixed + n_v * (n_v + 1) / 2;
+    }
+    const int64_t q0 = c->N - c->q; /* rows q0 .. N-1 attend t+1 keys each */
+    out[2] = (c->N * (c->N + 1) - q0 * (q0 + 1)) / 2;
+    return ORACLE_OK;
 }
 
 /* Exact softmax attention of row t, head h over the given keys ([APB-V-IT]

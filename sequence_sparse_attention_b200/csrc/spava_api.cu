@@ -763,24 +763,14 @@ constexpr size_t kNoAllocStatusBytes = 256;                // status word, then 
 
 static __device__ __align__(256) unsigned char g_score_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void *g_scratch_addr[kMaxDevices] = {};
-
 // Device address of g_score_scratch on the current device.  The name is only
-// a host-side stand-in for the array, so the address is looked up once per
-// device, with that device current.
+// a host-side stand-in for the array, so the address is looked up with the
+// device current, on every call: the lookup is cheap once the module is
+// loaded, and no address can outlive a reset of the device's context.
 spava_status scratch_address(void **out) {
-    int dev = 0;
-    SPAVA_CUDA(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= kMaxDevices) return SPAVA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        SPAVA_CUDA(cudaGetSymbolAddress(&p, g_score_scratch));
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    void *p = nullptr;
+    SPAVA_CUDA(cudaGetSymbolAddress(&p, g_score_scratch));
+    *out = p;
     return SPAVA_OK;
 }
 
@@ -842,4 +832,20 @@ extern "C" spava_status spava_score_noalloc(const spava_config *cfg, const void 
         score_kernel<64><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<64>::kAlloc, st>>>(p);
     }
     return launched();
+}
+
+extern "C" spava_status spava_score_noalloc_status(void *stream, int32_t *flags) {
+    if (!flags) return SPAVA_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    SPAVA_TRY(scratch_address(&scratch));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    SPAVA_CUDA(cudaMemcpyAsync(&h, scratch, sizeof(h), cudaMemcpyDeviceToHost, st));
+    SPAVA_CUDA(cudaStreamSynchronize(st));
+    if (h) {
+        SPAVA_CUDA(cudaMemsetAsync(scratch, 0, sizeof(h), st));
+        SPAVA_CUDA(cudaStreamSynchronize(st));
+    }
+    *flags = h;
+    return (h & kStatusTimeout) ? SPAVA_ERR_TIMEOUT : SPAVA_OK;
 }

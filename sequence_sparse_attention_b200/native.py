@@ -21,7 +21,7 @@ EXPORTS = ("spava_workspace_size", "spava_packed_len", "spava_score", "spava_top
            "spava_pack_passing", "spava_attn", "spava_prefill_attention",
            "spava_prefill_attention_host", "spava_device_status", "spava_attended_pairs",
            "spava_status_string", "spava_last_cuda_error", "spava_score_noalloc",
-           "spava_selftest_wait_timeout", "spava_plan_chunks")
+           "spava_selftest_wait_timeout", "spava_plan_chunks", "spava_score_noalloc_status")
 
 
 class SpavaConfig(ctypes.Structure):
@@ -75,6 +75,7 @@ def load() -> ctypes.CDLL:
         "spava_device_status": [vp, sz, vp, ctypes.POINTER(ctypes.c_int32)],
         "spava_attended_pairs": [cfgp, i64p, i64p],
         "spava_score_noalloc": [cfgp, vp, vp, vp, vp],
+        "spava_score_noalloc_status": [vp, ctypes.POINTER(ctypes.c_int32)],
         "spava_selftest_wait_timeout": [vp, sz, vp],
         "spava_plan_chunks": [ctypes.c_int32, i64p, ctypes.c_int64, ctypes.c_int64, i64p],
     }

@@ -56,6 +56,13 @@ class Workload:
     local_pair_full: int = 1
     score_norm: int = 0     # selection variants (see spava_config)
     score_pool: int = 0
+    # Uneven frames: token counts of the context's frames in order (the anchor
+    # and the query block count as one frame each); () = frames of `frame`
+    # tokens over absolute positions.
+    frame_tokens: tuple = ()
+    # Explicit chunk offsets off[0..2H], e.g. from the visual load balancer
+    # (spava_plan_chunks); () = the split chunk_offsets() draws.
+    offsets: tuple = ()
 
     @property
     def n_chunks(self) -> int:
@@ -87,6 +94,11 @@ WORKLOADS = {
 def chunk_offsets(w: Workload) -> np.ndarray:
     """Chunk boundaries ``off[0..2H]`` (int64): off[0] = a, off[2H] = N - q."""
     nc, C = w.n_chunks, w.context
+    if w.offsets:
+        off = np.asarray(w.offsets, dtype=np.int64)
+        if len(off) != nc + 1 or off[0] != w.a or off[-1] != w.N - w.q or (np.diff(off) < 1).any():
+            raise ValueError("explicit offsets do not split the context into 2H chunks")
+        return off
     if C < nc:
         raise ValueError("context shorter than the number of chunks")
     if w.jitter <= 0.0:
@@ -135,7 +147,14 @@ def make_inputs(w: Workload, device: str | torch.device = "cpu"):
     device = torch.device(device)
     g = torch.Generator(device=device).manual_seed(w.seed)
     Q = _randn_slabs(g, (w.N, w.Hq, w.d), device)
-    n_frames = (w.N + w.frame - 1) // w.frame
+    if w.frame_tokens:
+        if sum(w.frame_tokens) != w.context:
+            raise ValueError("frame_tokens must add up to the context length")
+        # frame boundaries: the anchor, each context frame, the query block
+        bounds = torch.tensor(np.cumsum([w.a] + list(w.frame_tokens) + [w.q]), device=device)
+        n_frames = len(w.frame_tokens) + 2
+    else:
+        n_frames = (w.N + w.frame - 1) // w.frame
     K = torch.empty((w.N, w.Hkv, w.d), dtype=torch.bfloat16, device=device)
     z = _randn_slabs(g, (w.N, w.Hkv, w.d), device)
     o = torch.randn((n_frames, w.Hkv, w.d), generator=g, device=device,
@@ -143,7 +162,8 @@ def make_inputs(w: Workload, device: str | torch.device = "cpu"):
     slab = 8192
     for t0 in range(0, w.N, slab):
         t1 = min(w.N, t0 + slab)
-        fr = torch.arange(t0, t1, device=device) // w.frame
+        pos = torch.arange(t0, t1, device=device)
+        fr = torch.bucketize(pos, bounds, right=True) if w.frame_tokens else pos // w.frame
         K[t0:t1] = (z[t0:t1].float() + o[fr]).to(torch.bfloat16)
     del z
     V = _randn_slabs(g, (w.N, w.Hkv, w.d), device)
@@ -153,6 +173,13 @@ def make_inputs(w: Workload, device: str | torch.device = "cpu"):
         pos = perm[: int(round(w.heavy_frac * C))] + w.a
         K[pos] = (K[pos].float() * w.heavy_mult).to(torch.bfloat16)
     return Q, K, V, chunk_offsets(w)
+
+
+def uneven_frames(n_frames: int, lo: int, hi: int, seed: int) -> tuple:
+    """Token counts of ``n_frames`` frames drawn uniformly from [lo, hi)
+    (seeded): frames of uneven resolution for the visual load balancer."""
+    g = torch.Generator().manual_seed(seed)
+    return tuple(int(x) for x in torch.randint(lo, hi, (n_frames,), generator=g))
 
 
 def bf16_bits(x: torch.Tensor) -> np.ndarray:

@@ -44,14 +44,21 @@ class OracleRun:
                                    self.idx if idx is None else idx, rows, heads)
 
 
-def check_selection(w: Workload, scores_oracle: np.ndarray, idx_gpu: np.ndarray, groups):
+def check_selection(w: Workload, scores_oracle: np.ndarray, idx_gpu: np.ndarray, groups,
+                    idx_oracle: np.ndarray | None = None) -> dict:
     """Every (chunk, group) selection is a valid top-l of the oracle scores (or
     of their window sums, with pooling): the same set wherever the l-th /
     (l+1)-th gap exceeds SEL_BAND relative, otherwise the same outside the band
-    around the l-th value."""
+    around the l-th value.
+
+    Returns counts for the record: ``exact`` selections decided by a clear gap
+    (or trivially: l = 0 or l >= n), ``band`` selections whose l-th and
+    (l+1)-th scores lie within the band, ``band_keys`` the number of keys
+    inside each such band, and ``differ`` the selections that are not the
+    oracle's own (possible only inside a band)."""
     scores_oracle = oracle.selection_scores(problem(w), scores_oracle)
     off = chunk_offsets(w)
-    n_exact = n_band = 0
+    rep = {"exact": 0, "band": 0, "band_keys": [], "differ": 0}
     for u in range(2 * w.H - 1):
         n = int(off[u + 1] - off[u])
         k = min(w.l, n)
@@ -62,8 +69,10 @@ def check_selection(w: Workload, scores_oracle: np.ndarray, idx_gpu: np.ndarray,
             sel = got[:k]
             assert (np.diff(sel) > 0).all(), (u, g, "not ascending")
             assert ((sel >= off[u]) & (sel < off[u + 1])).all(), (u, g, "outside chunk")
+            if idx_oracle is not None and not np.array_equal(got, idx_oracle[u, g]):
+                rep["differ"] += 1
             if k == 0 or k == n:
-                n_exact += 1
+                rep["exact"] += 1
                 continue
             S = scores_oracle[g, s0:s0 + n]
             srt = np.sort(S)[::-1]
@@ -73,56 +82,28 @@ def check_selection(w: Workload, scores_oracle: np.ndarray, idx_gpu: np.ndarray,
             if (sl - sl1) > SEL_BAND * abs(sl):
                 want = S >= sl
                 assert (chosen == want).all(), (u, g, "set differs with a clear gap")
-                n_exact += 1
+                rep["exact"] += 1
             else:
                 hi, lo = sl + SEL_BAND * abs(sl), sl - SEL_BAND * abs(sl)
                 assert chosen[S > hi].all(), (u, g, "missed a key above the band")
                 assert not chosen[S < lo].any(), (u, g, "took a key below the band")
-                n_band += 1
-    return n_exact, n_band
+                rep["band"] += 1
+                rep["band_keys"].append(int(((S >= lo) & (S <= hi)).sum()))
+    return rep
 
 
-def unique_mask(w: Workload, idx_gpu: np.ndarray, idx_ref: np.ndarray, rows, heads) -> np.ndarray:
-    """``[len(rows), len(heads)]``: True where the expected output does not
-    depend on how a tie in the selection was broken.
+def expected_rows(ref: "OracleRun", idx_gpu: np.ndarray, rows, heads, cached=None):
+    """The oracle's outputs for the GPU's own selection.
 
-    Two selections that both pass `check_selection` may differ among keys whose
-    scores tie within fp32 resolution.  A context row of chunk v reads the
-    passing blocks of chunks u < v of its KV group (the anchor and query rows
-    read none), so its output is unique only while the selections of every
-    such (u, g) agree.  The rows where they do not are checked with
-    `check_convex` instead."""
-    off = chunk_offsets(w)
-    G = w.Hq // w.Hkv
-    first_diff = np.full(w.Hkv, 2 * w.H, dtype=np.int64)
-    for g in range(w.Hkv):
-        for u in range(2 * w.H - 1):
-            if not np.array_equal(idx_gpu[u, g], idx_ref[u, g]):
-                first_diff[g] = u
-                break
-    rows = np.asarray(rows, dtype=np.int64)
-    v = np.searchsorted(off, rows, side="right") - 1       # chunk of each context row
-    context = (rows >= w.a) & (rows < w.N - w.q)
-    g_of = np.asarray(heads) // G
-    return ~context[:, None] | (v[:, None] <= first_diff[g_of][None, :])
-
-
-def check_convex(O_gpu: np.ndarray, V: torch.Tensor, heads, G: int, mask: np.ndarray, what=""):
-    """Outputs whose key set is one of several valid ones: each is a softmax
-    average of value rows of its KV group, so every coordinate lies within that
-    group's value range (plus bf16 rounding).  ``O_gpu[n, len(heads), d]``; the
-    entries where ``mask[n, len(heads)]`` is True are checked."""
-    Vf = V.float()
-    lo = Vf.amin(dim=0).cpu().numpy()        # [Hkv, d]
-    hi = Vf.amax(dim=0).cpu().numpy()
-    g_of = np.asarray(heads) // G
-    slack = 2.0 ** -7 * np.maximum(np.abs(lo), np.abs(hi))
-    lo_e = np.broadcast_to((lo - slack)[g_of][None], O_gpu.shape)[mask]
-    hi_e = np.broadcast_to((hi + slack)[g_of][None], O_gpu.shape)[mask]
-    got = O_gpu[mask]
-    assert np.isfinite(got).all(), f"{what}: non-finite output"
-    assert (got >= lo_e).all(), f"{what}: below the value range"
-    assert (got <= hi_e).all(), f"{what}: above the value range"
+    Once `check_selection` has accepted ``idx_gpu`` as a correct top-l (equal
+    to the oracle's wherever the scores leave no choice, inside the band where
+    they tie), every row has exactly one expected output: the oracle's
+    attention over the key set that selection gives.  Where the two
+    selections are identical that is the oracle's own result (``cached``, if
+    given, is returned)."""
+    if cached is not None and np.array_equal(idx_gpu, ref.idx):
+        return cached
+    return ref.rows(rows, heads, idx=idx_gpu)
 
 
 def check_outputs(O_gpu: np.ndarray, O_ref: np.ndarray, what=""):

@@ -171,23 +171,21 @@ def test_variant_configs_accepted_and_noalloc_refuses_row_norm():
     assert status("spava_score_noalloc", lay_of(w, score_norm=1), fake, fake, fake, None) == 2
 
 
-def test_plan_chunks_spreads_frames_evenly():
-    """Visual load balancing: consecutive whole frames, counts differing by at
-    most one with the extra frames in the first chunks; offsets accumulate the
-    frames' tokens from the anchor on, and form a valid layer."""
+def test_plan_chunks_matches_the_oracle():
+    """Visual load balancing: the library's chunk offsets equal the oracle's
+    (whole consecutive frames dealt evenly over the 2H virtual hosts) on random
+    frame lists, and form a valid layer."""
     from sequence_sparse_attention_b200.api import plan_chunks
     rng = np.random.default_rng(5)
-    for H, n_frames in ((1, 2), (2, 9), (4, 64), (8, 1006), (3, 37)):
-        ft = rng.integers(100, 300, n_frames)
-        off = plan_chunks(H, ft, 64)
-        nc = 2 * H
-        counts = [n_frames // nc + (1 if v < n_frames % nc else 0) for v in range(nc)]
-        bounds = np.concatenate([[0], np.cumsum(counts)])
-        want = 64 + np.concatenate([[0], np.cumsum(ft)])[bounds]
-        np.testing.assert_array_equal(off, want)
-        lay = Layout(H, 4, 2, 64, int(off[-1]) + 16, 64, 16, off, 8)
-        n = ctypes.c_size_t()
-        assert status("spava_workspace_size", lay, ctypes.byref(n)) == 0
+    for H, n_frames in ((1, 2), (2, 9), (4, 64), (8, 1006), (3, 37), (16, 1024), (32, 64)):
+        for trial in range(3):
+            ft = rng.integers(1 if trial == 0 else 100, 300, n_frames)
+            a = int(rng.integers(0, 2000))
+            off = plan_chunks(H, ft, a)
+            np.testing.assert_array_equal(off, oracle.plan_chunks(H, ft, a))
+            lay = Layout(H, 4, 2, 64, int(off[-1]) + 16, a, 16, off, 8)
+            n = ctypes.c_size_t()
+            assert status("spava_workspace_size", lay, ctypes.byref(n)) == 0
 
 
 def test_plan_chunks_equal_frames_divide_evenly():

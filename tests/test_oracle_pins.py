@@ -423,3 +423,69 @@ def test_variant_flags_are_validated():
         p.score_norm, p.score_pool = norm, pool
         with pytest.raises(ValueError):
             oracle.chunk_scores(p, Qb, Kb, 0, 0)
+
+
+def _compositions(n, k):
+    """Every way of writing n as an ordered sum of k positive integers."""
+    if k == 1:
+        yield (n,)
+        return
+    for first in range(1, n - k + 2):
+        for rest in _compositions(n - first, k - 1):
+            yield (first,) + rest
+
+
+@pytest.mark.parametrize("H,n_frames", [(1, 2), (1, 5), (2, 4), (2, 7), (2, 11), (3, 6), (3, 13)])
+def test_plan_chunks_brute_force(H, n_frames):
+    """Visual load balancing, pinned by enumeration: over EVERY split of the
+    frame list into 2H runs of consecutive whole frames, the ones whose frame
+    counts differ by at most one and never grow from one virtual host to the
+    next are a single split, and it is the oracle's; the offsets add up the
+    tokens of each run after the anchor."""
+    rng = np.random.default_rng(100 * H + n_frames)
+    ft = rng.integers(1, 50, n_frames)
+    nc = 2 * H
+    even = [c for c in _compositions(n_frames, nc)
+            if max(c) - min(c) <= 1 and all(c[v] >= c[v + 1] for v in range(nc - 1))]
+    assert len(even) == 1
+    counts = even[0]
+    a = int(rng.integers(0, 30))
+    want = [a]
+    f = 0
+    for c in counts:
+        want.append(want[-1] + int(sum(ft[f:f + c])))
+        f += c
+    np.testing.assert_array_equal(oracle.plan_chunks(H, ft, a), want)
+
+
+def test_plan_chunks_equal_frames_are_equal_chunks():
+    """Closed form: n_frames = 2H m frames of F tokens give chunks of m F tokens."""
+    off = oracle.plan_chunks(4, [256] * 64, 1024)
+    np.testing.assert_array_equal(off, 1024 + 256 * 8 * np.arange(9))
+
+
+@pytest.mark.parametrize("args", [(2, [5, 5, 5], 0), (1, [5, 0], 0), (1, [5, 5], -1), (0, [5, 5], 0)])
+def test_plan_chunks_rejects_impossible_splits(args):
+    with pytest.raises(ValueError):
+        oracle.plan_chunks(*args)
+
+
+@pytest.mark.parametrize("lpf", [0, 1])
+@pytest.mark.parametrize("H,a,l,jitter", [(1, 16, 4, 0.0), (2, 0, 7, 0.0), (3, 10, 5, 0.2),
+                                          (4, 9, 100, 0.0), (2, 12, 0, 0.3)])
+def test_attended_pairs_closed_form_counts_the_key_sets(lpf, H, a, l, jitter):
+    """The closed-form pair count equals the sizes of the key sets listed one
+    row at a time (any valid selection: every passing block has l_eff keys)."""
+    w = small(H=H, N=a + 8 + 2 * H * 32, a=a, q=8, l=l, frame=8, jitter=jitter,
+              local_pair_full=lpf)
+    p = problem(w)
+    off = chunk_offsets(w)
+    idx = np.full((2 * H - 1, w.Hkv, max(l, 1)), -1, dtype=np.int32)[:, :, :l]
+    for u in range(2 * H - 1):
+        k = min(l, int(off[u + 1] - off[u]))
+        idx[u, :, :k] = off[u] + np.arange(k)
+    counts = [0, 0, 0]
+    for t in range(w.N):
+        cls = 0 if t < w.a else (2 if t >= w.N - w.q else 1)
+        counts[cls] += len(oracle.key_set(p, idx, t, 0))
+    assert oracle.attended_pairs(p) == tuple(counts)

@@ -3,9 +3,11 @@ allocate device memory (a plug-in handed only its input and output buffers, or
 code that must not allocate after start-up).  Its scratch is a fixed array
 inside the library instead of a caller workspace.
 
-Called through the C ABI twice in a row, on two different layers, each result
-checked against spava_score with a workspace; a third layer that does not fit
-the fixed array must be refused before anything runs.
+Called through the C ABI twice in a row, on two different layers.  Each result
+must be bit-identical to spava_score with a workspace (the same kernels run in
+the same order) and match the oracle's scores; the status word of the fixed
+array must read clean after each call.  A third layer that does not fit the
+fixed array must be refused before anything runs.
 """
 import ctypes
 
@@ -13,10 +15,11 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import SCORE_REL
+import oracle
+from parity_util import SCORE_REL, problem
 from sequence_sparse_attention_b200 import native
 from sequence_sparse_attention_b200.api import Layout, Spava
-from sequence_sparse_attention_b200.synth import Workload, make_inputs
+from sequence_sparse_attention_b200.synth import Workload, bf16_bits, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -28,11 +31,13 @@ def scores_noalloc(w, Q, K):
     lay = Layout.from_workload(w)
     cfg = lay.c()
     out = torch.full((w.Hkv, lay.context), float("nan"), dtype=torch.float32, device="cuda")
-    rc = native.load().spava_score_noalloc(ctypes.byref(cfg), Q.data_ptr(), K.data_ptr(),
-                                           out.data_ptr(),
-                                           torch.cuda.current_stream().cuda_stream)
+    stream = torch.cuda.current_stream().cuda_stream
+    lib = native.load()
+    rc = lib.spava_score_noalloc(ctypes.byref(cfg), Q.data_ptr(), K.data_ptr(), out.data_ptr(), stream)
     assert rc == 0, native.STATUS_NAMES.get(rc, rc)
-    torch.cuda.synchronize()
+    flags = ctypes.c_int32(-1)
+    rc = lib.spava_score_noalloc_status(stream, ctypes.byref(flags))
+    assert rc == 0 and flags.value == 0, (rc, flags.value)
     return out
 
 
@@ -47,12 +52,14 @@ def scores_with_workspace(w, Q, K):
 def test_noalloc_scores_match_workspace_scores_on_two_calls():
     for w in (FIRST, SECOND):
         Q, K, _, off = make_inputs(w)
-        Q, K = Q.cuda(), K.cuda()
         last0 = int(off[-2] - w.a)      # columns of the producing chunks
-        got = scores_noalloc(w, Q, K)[:, :last0].cpu().numpy()
-        want = scores_with_workspace(w, Q, K)[:, :last0].cpu().numpy()
+        got = scores_noalloc(w, Q.cuda(), K.cuda())[:, :last0].cpu().numpy()
+        want = scores_with_workspace(w, Q.cuda(), K.cuda())[:, :last0].cpu().numpy()
         assert np.isfinite(got).all()
-        np.testing.assert_allclose(got, want, rtol=SCORE_REL, atol=0)
+        np.testing.assert_array_equal(got, want)   # same kernels, same order: same bits
+        ref, _ = oracle.scores_and_select(problem(w), bf16_bits(Q), bf16_bits(K))
+        np.testing.assert_allclose(got, ref[:, :last0], rtol=SCORE_REL,
+                                   atol=1e-7 * w.q * w.Hq / w.Hkv)
 
 
 def test_noalloc_refuses_layers_beyond_the_fixed_scratch():
