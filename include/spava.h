@@ -205,6 +205,86 @@ spava_status spava_attended_pairs(const spava_config *cfg, int64_t pairs[3], int
 spava_status spava_plan_chunks(int32_t H, const int64_t *frame_tokens, int64_t n_frames,
                                int64_t anchor_len, int64_t *chunk_offsets);
 
+/* ---------------------------------------------------------------------------
+ * Multi-GPU ZigZag sequence parallelism ("Riepilogo Tecnico: APB-V",
+ * Metodologia, "Suddivisione del Contesto e Disposizione ZigZag": physical host
+ * p holds virtual hosts p and 2H-1-p; Ottimizzazioni a Livello di Sistema,
+ * "Comunicazione Sovrapposta": the passing blocks travel between hosts while
+ * the hosts compute, and "Forward Fuso di Contesto e Query": the query rows'
+ * partial results of every host are merged through their log-sum-exp).
+ *
+ * `world` GPUs, one process each; H % world == 0.  Rank r holds the physical
+ * hosts p in [r*m, (r+1)*m), m = H/world -- the chunks v with
+ * pair(v) / m == r, pair(v) = v < H ? v : 2H-1-v -- plus the anchor and the
+ * query block, which every rank holds.  Its token-major buffers (q, k, v, o:
+ * [n_local, heads, d]; lse: [Hq, n_local]) are LOCAL: [anchor | its chunks in
+ * increasing v | query block].  A rank computes its chunks' context rows, and
+ * (like every rank) the anchor rows and the query rows.
+ *
+ * One layer on each rank, in this order (all on `stream`, asynchronous):
+ *   spava_shard_front        scores, top-l and gather of its chunks' passing
+ *                            blocks; writes its pass message
+ *   all-gather #1            the caller gathers every rank's pass message,
+ *                            rank-major, into pass_all (e.g. NCCL
+ *                            all-gather into this GPU's own memory)
+ *   spava_shard_local_attn   anchor rows and the query rows' partials over
+ *                            the anchor, its chunks and the query block: needs
+ *                            nothing from other ranks, so it runs while
+ *                            all-gather #1 is in flight; writes its part message
+ *   all-gather #2            every rank's part message into part_all
+ *   spava_shard_context_attn unpacks pass_all, then the context rows of its
+ *                            chunks (runs while all-gather #2 is in flight)
+ *   spava_shard_merge        unpacks part_all, merges the query rows
+ * The messages have the same size on every rank (spava_shard_sizes).  The
+ * outputs equal spava_prefill_attention's rows bit for bit.  score_norm 1 is
+ * not offered (SPAVA_ERR_UNSUPPORTED): it needs every chunk's statistics of the
+ * query rows before scoring.  The same workspace serves all four calls of a
+ * rank; the caller keeps pass_send / part_send unchanged until its gathers
+ * have read them.
+ * ------------------------------------------------------------------------- */
+
+/* Host only.  local_first (HOST [2H+2], may be NULL): first local row of the
+ * anchor (index 0), chunk v (1+v), the query block (2H+1), -1 where the rank
+ * does not hold the region; *n_local: rows of its local buffers; slot_chunk
+ * (HOST [2H/world], may be NULL): the chunk in each slot of its messages.
+ * SPAVA_ERR_INVALID_ARG for rank outside [0, world) or world < 1,
+ * SPAVA_ERR_UNSUPPORTED if world does not divide H or score_norm is 1. */
+spava_status spava_shard_layout(const spava_config *cfg, int32_t rank, int32_t world,
+                                int64_t *local_first, int64_t *n_local, int32_t *slot_chunk);
+
+/* Host only: workspace bytes of a rank (256-byte aligned buffer, first 256
+ * bytes the status block as for spava_workspace_size), and the bytes of one
+ * rank's pass and part messages (pass_all / part_all hold world of each). */
+spava_status spava_shard_sizes(const spava_config *cfg, int32_t world, size_t *ws_bytes,
+                               size_t *pass_msg_bytes, size_t *part_msg_bytes);
+
+/* Reads local q, k, v; writes pass_send (device, 16-byte aligned,
+ * pass_msg_bytes): per slot the indices and the K and V rows of that chunk's
+ * passing block. */
+spava_status spava_shard_front(const spava_config *cfg, int32_t rank, int32_t world, const void *q,
+                               const void *k, const void *v, void *pass_send, void *ws,
+                               size_t ws_bytes, void *stream);
+
+/* Writes the anchor rows of o / lse and part_send (device, part_msg_bytes):
+ * the query rows' partials over this rank's chunks. */
+spava_status spava_shard_local_attn(const spava_config *cfg, int32_t rank, int32_t world,
+                                    const void *q, const void *k, const void *v, void *o, float *lse,
+                                    void *part_send, void *ws, size_t ws_bytes, void *stream);
+
+/* Reads pass_all (device, world * pass_msg_bytes, rank-major); writes the
+ * context rows of this rank's chunks into o / lse, and, if idx_out != NULL,
+ * every chunk's passing-block indices [2H-1, Hkv, l]. */
+spava_status spava_shard_context_attn(const spava_config *cfg, int32_t rank, int32_t world,
+                                      const void *q, const void *k, const void *v,
+                                      const void *pass_all, void *o, float *lse, int32_t *idx_out,
+                                      void *ws, size_t ws_bytes, void *stream);
+
+/* Reads part_all (device, world * part_msg_bytes, rank-major); writes the
+ * query rows of o / lse. */
+spava_status spava_shard_merge(const spava_config *cfg, int32_t rank, int32_t world,
+                               const void *part_all, void *o, float *lse, void *ws, size_t ws_bytes,
+                               void *stream);
+
 /* spava_score for callers that cannot allocate device memory: same inputs,
  * same scores output, no workspace argument.  (The pages have no counterpart:
  * this is an interface choice of the library, not part of the method.)

@@ -204,3 +204,142 @@ class Spava:
         lib.spava_device_status(_ptr(self.ws), self.ws.numel(), _stream(self.device),
                                 ctypes.byref(flags))
         return flags.value
+
+
+# ------------------------------------------------------------------ shards
+def shard_layout(lay: Layout, rank: int, world: int):
+    """Local layout of rank ``rank`` of ``world``: (first local row of each
+    region [2H+2] -- anchor, chunk 0..2H-1, query block; -1 if not held --,
+    rows of the local buffers, the chunks of its message slots)."""
+    first = np.empty(2 * lay.H + 2, dtype=np.int64)
+    n_local = ctypes.c_int64()
+    m = lay.H // world if world > 0 and lay.H % world == 0 else 0
+    slots = np.empty(max(1, 2 * m), dtype=np.int32)
+    cfg = lay.c()
+    P = ctypes.POINTER
+    native.call("spava_shard_layout", ctypes.byref(cfg), int(rank), int(world),
+                first.ctypes.data_as(P(ctypes.c_int64)), ctypes.byref(n_local),
+                slots.ctypes.data_as(P(ctypes.c_int32)))
+    return first, n_local.value, slots[:2 * m].copy()
+
+
+def shard_sizes(lay: Layout, world: int):
+    """(workspace bytes, pass message bytes, partial message bytes) per rank."""
+    ws, pm, qm = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    cfg = lay.c()
+    native.call("spava_shard_sizes", ctypes.byref(cfg), int(world), ctypes.byref(ws),
+                ctypes.byref(pm), ctypes.byref(qm))
+    return ws.value, pm.value, qm.value
+
+
+def local_positions(lay: Layout, first: np.ndarray) -> np.ndarray:
+    """Global token position of every local row, from a shard layout."""
+    off = np.asarray(lay.offsets, dtype=np.int64)
+    bounds = [(0, lay.a)] + [(int(off[v]), int(off[v + 1])) for v in range(2 * lay.H)] + \
+             [(lay.N - lay.q, lay.N)]
+    parts = [None] * len(bounds)
+    for r, (lo, hi) in enumerate(bounds):
+        if first[r] >= 0:
+            parts[r] = (int(first[r]), np.arange(lo, hi, dtype=np.int64))
+    held = sorted((p for p in parts if p is not None), key=lambda x: x[0])
+    return np.concatenate([x for _, x in held]) if held else np.zeros(0, dtype=np.int64)
+
+
+class SpavaShard:
+    """One rank of the ZigZag sequence-parallel layer: rank ``rank`` of
+    ``world`` GPUs holds the physical hosts p in [rank*m, (rank+1)*m),
+    m = H/world (chunks p and 2H-1-p of each), in local buffers laid out
+    [anchor | its chunks in increasing order | query block].  The two
+    exchanges -- every rank's passing blocks, every rank's query-row partials
+    -- are all-gathers of fixed-size byte messages between the calls."""
+
+    def __init__(self, lay: Layout, rank: int, world: int, device="cuda"):
+        self.lay, self.rank, self.world = lay, rank, world
+        self.device = torch.device(device)
+        self.cfg = lay.c()
+        self.first, self.n_local, self.slots = shard_layout(lay, rank, world)
+        self.positions = local_positions(lay, self.first)
+        ws, pm, qm = shard_sizes(lay, world)
+        self.ws = torch.zeros(ws, dtype=torch.uint8, device=self.device)
+        self.pass_send = torch.zeros(pm, dtype=torch.uint8, device=self.device)
+        self.part_send = torch.zeros(qm, dtype=torch.uint8, device=self.device)
+        self.pass_all = torch.zeros(world * pm, dtype=torch.uint8, device=self.device)
+        self.part_all = torch.zeros(world * qm, dtype=torch.uint8, device=self.device)
+
+    def _args(self):
+        return ctypes.byref(self.cfg), int(self.rank), int(self.world)
+
+    def check_local(self, q, k, v=None):
+        lay = self.lay
+        _check(q, (self.n_local, lay.Hq, lay.d), torch.bfloat16, "q")
+        _check(k, (self.n_local, lay.Hkv, lay.d), torch.bfloat16, "k")
+        if v is not None:
+            _check(v, (self.n_local, lay.Hkv, lay.d), torch.bfloat16, "v")
+
+    def front(self, q, k, v):
+        self.check_local(q, k, v)
+        native.call("spava_shard_front", *self._args(), _ptr(q), _ptr(k), _ptr(v),
+                    _ptr(self.pass_send), _ptr(self.ws), self.ws.numel(), _stream(self.device))
+
+    def check_out(self, o, lse):
+        lay = self.lay
+        _check(o, (self.n_local, lay.Hq, lay.d), torch.bfloat16, "o")
+        if lse is not None:
+            _check(lse, (lay.Hq, self.n_local), torch.float32, "lse")
+
+    def local_attn(self, q, k, v, o, lse):
+        self.check_local(q, k, v)
+        self.check_out(o, lse)
+        native.call("spava_shard_local_attn", *self._args(), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                    _ptr(lse), _ptr(self.part_send), _ptr(self.ws), self.ws.numel(),
+                    _stream(self.device))
+
+    def context_attn(self, q, k, v, o, lse, idx_out=None):
+        self.check_local(q, k, v)
+        self.check_out(o, lse)
+        if idx_out is not None:
+            lay = self.lay
+            _check(idx_out, (2 * lay.H - 1, lay.Hkv, lay.l), torch.int32, "idx_out")
+        native.call("spava_shard_context_attn", *self._args(), _ptr(q), _ptr(k), _ptr(v),
+                    _ptr(self.pass_all), _ptr(o), _ptr(lse), _ptr(idx_out), _ptr(self.ws),
+                    self.ws.numel(), _stream(self.device))
+
+    def merge(self, o, lse):
+        self.check_out(o, lse)
+        native.call("spava_shard_merge", *self._args(), _ptr(self.part_all), _ptr(o), _ptr(lse),
+                    _ptr(self.ws), self.ws.numel(), _stream(self.device))
+
+    def new_outputs(self, want_lse=True):
+        lay = self.lay
+        o = torch.empty((self.n_local, lay.Hq, lay.d), dtype=torch.bfloat16, device=self.device)
+        lse = (torch.empty((lay.Hq, self.n_local), dtype=torch.float32, device=self.device)
+               if want_lse else None)
+        return o, lse
+
+    def layer(self, q, k, v, o, lse, all_gather, comm_stream=None, idx_out=None):
+        """One sharded layer.  ``all_gather(out, inp)`` gathers every rank's
+        ``inp`` bytes into ``out`` (rank-major) on the current stream, e.g.
+        ``torch.distributed.all_gather_into_tensor``.  With ``comm_stream``
+        the gathers run there: the passing blocks travel while this rank's
+        anchor rows and query partials compute, the partials while its
+        context rows compute."""
+        cur = torch.cuda.current_stream(self.device)
+        cs = comm_stream or cur
+        self.front(q, k, v)
+        if cs is not cur:
+            cs.wait_stream(cur)
+        with torch.cuda.stream(cs):
+            all_gather(self.pass_all, self.pass_send)
+        e_pass = cs.record_event() if cs is not cur else None
+        self.local_attn(q, k, v, o, lse)
+        if cs is not cur:
+            cs.wait_stream(cur)
+        with torch.cuda.stream(cs):
+            all_gather(self.part_all, self.part_send)
+        e_part = cs.record_event() if cs is not cur else None
+        if e_pass is not None:
+            cur.wait_event(e_pass)
+        self.context_attn(q, k, v, o, lse, idx_out)
+        if e_part is not None:
+            cur.wait_event(e_part)
+        self.merge(o, lse)

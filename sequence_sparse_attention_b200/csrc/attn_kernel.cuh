@@ -152,6 +152,7 @@ struct ItemPlan {
     Item it;
     int hB;  // query head of tile B
     int r0A, eA, r0B, eB;
+    int rs;  // global position minus local row of the item's rows
     bool hasB;
     Seg segs[kMaxSegs];
     int ns, T, TA, TB, g;
@@ -163,6 +164,7 @@ __device__ __forceinline__ void plan_item(const Layer &L, const Group *groups, i
     ip.it = decode_pair_item(groups, n_groups, b, L.G, &h_b);
     item_rows(L, ip.it, ip.r0A, ip.eA);
     ip.g = ip.it.h / L.G;
+    ip.rs = region_shift(L, item_region(L, ip.it));
     if (h_b != ip.it.h) {
         // Cross-head item (or a tile alone): B has A's rows and key sequence.
         ip.hasB = h_b >= 0;
@@ -293,11 +295,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         if (lane == 0) {
             mbar_expect_tx(q_full, hasB ? 2 * SM::kTile : SM::kTile);
             for (int p = 0; p < SM::kPanels; ++p)
-                tma_load_3d(smem + SM::kOffQ + p * 16384, &P.tmQ, p * 64, it.h, r0A, q_full);
+                tma_load_3d(smem + SM::kOffQ + p * 16384, &P.tmQ, p * 64, it.h, r0A - ip.rs, q_full);
             if (hasB)
                 for (int p = 0; p < SM::kPanels; ++p)
-                    tma_load_3d(smem + SM::kOffQ + SM::kTile + p * 16384, &P.tmQ, p * 64, ip.hB, r0B,
-                                q_full);
+                    tma_load_3d(smem + SM::kOffQ + SM::kTile + p * 16384, &P.tmQ, p * 64, ip.hB,
+                                r0B - ip.rs, q_full);
             int k_last[KS], v_last[VS];
             for (int i = 0; i < KS; ++i) k_last[i] = -1;
             for (int i = 0; i < VS; ++i) v_last[i] = -1;
@@ -312,7 +314,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 const int key0 = s.begin + kc.tile * kKeyTile;
                 for (int p = 0; p < SM::kPanels; ++p) {
                     if (s.src == 0)
-                        tma_load_3d(kd + p * 16384, &P.tmK, p * 64, g, key0, &k_full[ks]);
+                        tma_load_3d(kd + p * 16384, &P.tmK, p * 64, g, key0 - s.shift, &k_full[ks]);
                     else
                         tma_load_3d(kd + p * 16384, &P.tmPK, p * 64, key0, g, &k_full[ks]);
                 }
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 const int key0 = s.begin + vc.tile * kKeyTile;
                 for (int p = 0; p < SM::kPanels; ++p) {
                     if (s.src == 0)
-                        tma_load_3d(vd + p * 16384, &P.tmV, p * 64, g, key0, &v_full[vs]);
+                        tma_load_3d(vd + p * 16384, &P.tmV, p * 64, g, key0 - s.shift, &v_full[vs]);
                     else
                         tma_load_3d(vd + p * 16384, &P.tmPV, p * 64, key0, g, &v_full[vs]);
                 }
@@ -560,7 +562,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                     }
                     if (valid) P.part_lse[(static_cast<size_t>(it.sub) * L.Hq + hx) * L.q + i] = lse2;
                 } else {
-                    __nv_bfloat16 *dst = P.O + (static_cast<size_t>(t) * L.Hq + hx) * D;
+                    const int tl = t - ip.rs;  // local row
+                    __nv_bfloat16 *dst = P.O + (static_cast<size_t>(tl) * L.Hq + hx) * D;
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t u[32];
@@ -579,7 +582,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                             }
                         }
                     }
-                    if (valid && P.lse) P.lse[static_cast<size_t>(hx) * L.N + t] = lse2 * 0.69314718055994531f;
+                    if (valid && P.lse) P.lse[static_cast<size_t>(hx) * L.Nl + tl] = lse2 * 0.69314718055994531f;
                 }
             }
         }

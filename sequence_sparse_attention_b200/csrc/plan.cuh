@@ -22,6 +22,14 @@
 //     s = 0 anchor [0,a), s = 1+v chunk v, s = 2H+1 query block [N-q, t];
 //     the partials are merged by log-sum-exp afterwards.
 //   score statistics of chunk u: K [off[u], off[u+1]) for the query rows.
+//
+// Positions are global token positions throughout.  The token-major buffers
+// (Q, K, V, O, lse) may hold only some regions of the sequence -- a shard of
+// the ZigZag sequence parallelism holds the anchor, its own chunks and the
+// query block ("Comunicazione Sovrapposta": one physical host per GPU) -- laid
+// out region after region; Layer::loc gives each region's first local row,
+// and every load or store of a token row subtracts its region's shift.  On one
+// GPU every region is held at its global position (all shifts 0).
 #pragma once
 
 #include <stdint.h>
@@ -37,14 +45,28 @@ constexpr int kMaxPool = 255;    // widest score-pooling window
 
 enum ItemKind : int32_t { kCtx = 0, kAnchor = 1, kQueryPart = 2, kStats = 3 };
 
+// Regions of the sequence: 0 the anchor, 1 + v chunk v, 2H + 1 the query block.
+constexpr int kMaxRegions = kMaxChunks + 2;
+
 struct Layer {
     int32_t H, Hq, Hkv, d, G, lpf, l, n_chunks;
     int32_t norm, pool;                // selection variants: row-normalised scores, window width
     int32_t N, a, q, C, L;             // tokens, anchor, query, context, packed rows
+    int32_t Nl;                        // rows of the (local) token-major buffers
     float scale_log2;                  // softmax scale * log2(e)
+    uint64_t own;                      // bit v: chunk v is held (and computed) here
     int32_t off[kMaxChunks + 1];       // chunk offsets
     int32_t pcum[kMaxChunks + 1];      // packed row where P_u starts; pcum[0] = a
+    int32_t loc[kMaxRegions];          // first local row of each region, -1 if not held
 };
+
+__host__ __device__ inline int region_first(const Layer &L, int r) {
+    return r == 0 ? 0 : (r <= L.n_chunks ? L.off[r - 1] : L.N - L.q);
+}
+// Global position minus local row, for the rows of region r.
+__host__ __device__ inline int region_shift(const Layer &L, int r) { return region_first(L, r) - L.loc[r]; }
+__host__ __device__ inline int query_region(const Layer &L) { return L.n_chunks + 1; }
+__host__ __device__ inline bool owns(const Layer &L, int v) { return (L.own >> v) & 1u; }
 
 // A run of work items of one kind and one chunk/segment.  Items inside a group
 // are ordered (KV head, row tile descending, query head of that KV head): the
@@ -60,6 +82,7 @@ struct Item {
 
 struct Seg {
     int32_t src, begin, end, causal;
+    int32_t shift;  // src 0: global position minus local row of this segment's keys
 };
 
 __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
@@ -99,14 +122,23 @@ __host__ __device__ inline void item_rows(const Layer &L, const Item &it, int &r
     row_end = row0 + kRowTile < hi ? row0 + kRowTile : hi;
 }
 
-__host__ __device__ inline void add_seg(Seg *s, int &n, int src, int b, int e, int causal) {
+// Segment [b, e) of the packed passing K/V (src 1), or of region r's token
+// rows (src 0).
+__host__ __device__ inline void add_seg(const Layer &L, Seg *s, int &n, int src, int b, int e,
+                                        int causal, int region = 0) {
     if (e > b) {
         s[n].src = src;
         s[n].begin = b;
         s[n].end = e;
         s[n].causal = causal;
+        s[n].shift = src == 0 ? region_shift(L, region) : 0;
         ++n;
     }
+}
+
+// Region whose rows an item computes.
+__host__ __device__ inline int item_region(const Layer &L, const Item &it) {
+    return it.kind == kCtx ? 1 + it.sub : (it.kind == kAnchor ? 0 : query_region(L));
 }
 
 // Segments of the item's key sequence (at most kMaxSegs).  Returns their count.
@@ -118,30 +150,30 @@ __host__ __device__ inline int build_segments(const Layer &L, const Item &it, Se
             const int v = it.sub;
             if (L.lpf && v >= L.H) {
                 const int p = 2 * L.H - 1 - v;
-                add_seg(s, n, 1, 0, L.pcum[p], 0);
-                add_seg(s, n, 1, L.pcum[p + 1], L.pcum[v], 0);
-                add_seg(s, n, 0, L.off[p], L.off[p + 1], 0);
+                add_seg(L, s, n, 1, 0, L.pcum[p], 0);
+                add_seg(L, s, n, 1, L.pcum[p + 1], L.pcum[v], 0);
+                add_seg(L, s, n, 0, L.off[p], L.off[p + 1], 0, 1 + p);
             } else {
-                add_seg(s, n, 1, 0, L.pcum[v], 0);
+                add_seg(L, s, n, 1, 0, L.pcum[v], 0);
             }
-            add_seg(s, n, 0, L.off[v], row_end, 1);
+            add_seg(L, s, n, 0, L.off[v], row_end, 1, 1 + v);
             break;
         }
         case kAnchor:
-            add_seg(s, n, 0, 0, row_end, 1);
+            add_seg(L, s, n, 0, 0, row_end, 1, 0);
             break;
         case kQueryPart: {
             const int sg = it.sub;
             if (sg == 0)
-                add_seg(s, n, 0, 0, L.a, 0);
+                add_seg(L, s, n, 0, 0, L.a, 0, 0);
             else if (sg <= L.n_chunks)
-                add_seg(s, n, 0, L.off[sg - 1], L.off[sg], 0);
+                add_seg(L, s, n, 0, L.off[sg - 1], L.off[sg], 0, sg);
             else
-                add_seg(s, n, 0, L.N - L.q, row_end, 1);
+                add_seg(L, s, n, 0, L.N - L.q, row_end, 1, query_region(L));
             break;
         }
         default:  // kStats
-            add_seg(s, n, 0, L.off[it.sub], L.off[it.sub + 1], 0);
+            add_seg(L, s, n, 0, L.off[it.sub], L.off[it.sub + 1], 0, 1 + it.sub);
             break;
     }
     return n;

@@ -115,14 +115,15 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
         if (lane == 0) {
             mbar_expect_tx(a_full, SM::kTile);
             for (int p = 0; p < SM::kPanels; ++p)
-                tma_load_3d(smem + SM::kOffK + p * 16384, &P.tmK, p * 64, g, key0, a_full);
+                tma_load_3d(smem + SM::kOffK + p * 16384, &P.tmK, p * 64, g, key0 - region_shift(L, 1 + u),
+                            a_full);
             int q_last[QS];
             for (int i = 0; i < QS; ++i) q_last[i] = -1;
             for (int b = 0; b < NBLK; ++b) {
                 const int qs = b % QS;
                 if (b >= QS && !mbar_wait(&q_empty[qs], ((b / QS) - 1) & 1, ab)) break;
                 const int h = g * L.G + b / n_rb;
-                const int r0 = L.N - L.q + (b % n_rb) * 128;
+                const int r0 = L.N - L.q + (b % n_rb) * 128 - region_shift(L, query_region(L));
                 mbar_expect_tx(&q_full[qs], SM::kTile);
                 for (int p = 0; p < SM::kPanels; ++p)
                     tma_load_3d(smem + SM::kOffQ + qs * SM::kTile + p * 16384, &P.tmQ, p * 64, h, r0,

@@ -142,12 +142,21 @@ __device__ __forceinline__ int select_chunk(const Layer &L, const float *scores,
     return l_eff;
 }
 
-__global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, const float *scores,
-                                                              int32_t *idx) {
-    select_chunk(L, scores, idx, blockIdx.x / L.Hkv, blockIdx.x % L.Hkv);
+// The k-th producing chunk (u < 2H-1) held here, in increasing u; -1 if there
+// is none (the host sizes the grids so that there always is).
+__device__ __forceinline__ int nth_owned_producer(const Layer &L, int k) {
+    for (int u = 0; u < L.n_chunks - 1; ++u)
+        if (owns(L, u) && k-- == 0) return u;
+    return -1;
 }
 
-// Copies packed rows [r0, r1) of KV head g from the token rows src(r): one warp
+__global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, const float *scores,
+                                                              int32_t *idx) {
+    const int u = nth_owned_producer(L, blockIdx.x / L.Hkv);
+    if (u >= 0) select_chunk(L, scores, idx, u, blockIdx.x % L.Hkv);
+}
+
+// Copies packed rows [r0, r1) of KV head g from the local token rows src(r): one warp
 // per row, lanes 0-15 the K row and lanes 16-31 the V row in 16-byte pieces,
 // 8 rows in flight per warp.
 template <int D, typename Src>
@@ -177,36 +186,40 @@ __device__ __forceinline__ void copy_rows(const Layer &L, const __nv_bfloat16 *K
 }
 
 // Selection and gather in one launch (the layer entry points): CTA (u, g) for
-// u < 2H-1 selects the passing block of chunk u for KV head g exactly as
-// topk_kernel, then copies those K/V rows to the packed rows pcum[u] + r; the
-// CTAs after them copy the anchor rows.  The selected indices are read back
-// from idx by the CTA that wrote them (visible after __syncthreads).
+// each producing chunk u < 2H-1 held here selects the passing block of chunk u
+// for KV head g exactly as topk_kernel, then copies those K/V rows to the
+// packed rows pcum[u] + r; the CTAs after them copy the anchor rows.  The
+// selected indices are read back from idx by the CTA that wrote them (visible
+// after __syncthreads).
 constexpr int kAnchorRowsPerCta = 256;
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) select_pack_kernel(
     const Layer L, const float *scores, int32_t *idx, const __nv_bfloat16 *K,
-    const __nv_bfloat16 *V, __nv_bfloat16 *PK, __nv_bfloat16 *PV) {
-    const int n_sel = (L.n_chunks - 1) * L.Hkv;
+    const __nv_bfloat16 *V, __nv_bfloat16 *PK, __nv_bfloat16 *PV, int n_sel_ctas) {
+    const int n_sel = n_sel_ctas;
     const int warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
     if (static_cast<int>(blockIdx.x) < n_sel) {
-        const int u = blockIdx.x / L.Hkv, g = blockIdx.x % L.Hkv;
+        const int u = nth_owned_producer(L, blockIdx.x / L.Hkv), g = blockIdx.x % L.Hkv;
+        if (u < 0) return;
         const int l_eff = select_chunk(L, scores, idx, u, g);
         __syncthreads();
         const int32_t *sel = idx + (static_cast<size_t>(u) * L.Hkv + g) * L.l;
-        const int p0 = L.pcum[u];
+        const int p0 = L.pcum[u], sh = region_shift(L, 1 + u);
         copy_rows<D>(L, K, V, PK, PV, g, p0, p0 + l_eff, warp, n_warps,
-                     [&](int r) { return sel[r - p0]; });
+                     [&](int r) { return sel[r - p0] - sh; });
     } else {
         const int b = blockIdx.x - n_sel;
         const int per_g = (L.a + kAnchorRowsPerCta - 1) / kAnchorRowsPerCta;
         const int g = b / per_g, r0 = (b % per_g) * kAnchorRowsPerCta;
         const int r1 = min(L.a, r0 + kAnchorRowsPerCta);
-        copy_rows<D>(L, K, V, PK, PV, g, r0, r1, warp, n_warps, [](int r) { return r; });
+        const int sh = region_shift(L, 0);
+        copy_rows<D>(L, K, V, PK, PV, g, r0, r1, warp, n_warps, [&](int r) { return r - sh; });
     }
 }
 
 // Packed passing K/V: packed row `row` = g*L + r of KV head g is the anchor row r
-// (r < a) or the s-th kept key of chunk u (r = pcum[u] + s).  HBM-bound gather:
+// (r < a) or the s-th kept key of chunk u (r = pcum[u] + s); the rows of chunks
+// not held here are left alone.  HBM-bound gather:
 // persistent warps walk groups of 32 packed rows; lane i resolves the source of
 // row i with one coalesced index load, the sources are shuffled out, and rows are
 // copied 8 at a time (first half-warp K, second half V, 16 bytes per lane) with
@@ -214,11 +227,15 @@ __global__ void __launch_bounds__(kSelectThreads) select_pack_kernel(
 constexpr int kPackThreads = 256;
 constexpr int kPackBatch = 8;
 
+// Local token row of packed row r of KV head g; -1: a row to zero (an index
+// that is not a position of chunk u); -2: a row of a chunk not held here.
 __device__ __forceinline__ int packed_source(const Layer &L, const int32_t *idx, int g, int r) {
-    if (r < L.a) return r;
+    if (r < L.a) return r - region_shift(L, 0);
     int u = 0;
     while (u + 1 < L.n_chunks - 1 && r >= L.pcum[u + 1]) ++u;
-    return idx[(static_cast<size_t>(u) * L.Hkv + g) * L.l + (r - L.pcum[u])];
+    if (!owns(L, u)) return -2;
+    const int t = idx[(static_cast<size_t>(u) * L.Hkv + g) * L.l + (r - L.pcum[u])];
+    return (t >= L.off[u] && t < L.off[u + 1]) ? t - region_shift(L, 1 + u) : -1;
 }
 
 template <int D>
@@ -238,25 +255,27 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const Layer L, const
         // Source element offset of this lane's row, or -1 (past the end, or an
         // index that is not a token position: written as a zero row).
         const long long row_l = grp * 32 + lane;
-        long long src_l = -1;
+        long long src_l = -2;
         if (row_l < total) {
             const int g = static_cast<int>(row_l / L.L);
             const int src = packed_source(L, idx, g, static_cast<int>(row_l % L.L));
-            if (src >= 0 && src < L.N) src_l = (static_cast<long long>(src) * L.Hkv + g) * D;
+            src_l = src >= 0 ? (static_cast<long long>(src) * L.Hkv + g) * D : src;
         }
 #pragma unroll 1
         for (int b = 0; b < 32; b += kPackBatch) {
             uint4 v[kPackBatch];
+            long long so[kPackBatch];
 #pragma unroll
             for (int k = 0; k < kPackBatch; ++k) {
-                const long long so = __shfl_sync(0xffffffffu, src_l, b + k);
+                so[k] = __shfl_sync(0xffffffffu, src_l, b + k);
                 v[k] = make_uint4(0, 0, 0, 0);
-                if (so >= 0 && c < kChunks) v[k] = __ldg(reinterpret_cast<const uint4 *>(src_base + so) + c);
+                if (so[k] >= 0 && c < kChunks) v[k] = __ldg(reinterpret_cast<const uint4 *>(src_base + so[k]) + c);
             }
 #pragma unroll
             for (int k = 0; k < kPackBatch; ++k) {
                 const long long row = grp * 32 + b + k;
-                if (row < total && c < kChunks) reinterpret_cast<uint4 *>(dst_base + row * D)[c] = v[k];
+                if (row < total && so[k] != -2 && c < kChunks)
+                    reinterpret_cast<uint4 *>(dst_base + row * D)[c] = v[k];
             }
         }
     }
@@ -293,14 +312,14 @@ __global__ void __launch_bounds__(256) merge_kernel(const Layer L, const float *
         }
     }
     const float inv = 1.f / wsum;
-    const int t = L.N - L.q + i;
+    const int t = L.N - L.q + i - region_shift(L, query_region(L));  // local row
     if (lane < D / 4) {
         uint2 v;
         v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
         v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
         reinterpret_cast<uint2 *>(O + (static_cast<size_t>(t) * L.Hq + h) * D)[lane] = v;
     }
-    if (lane == 0 && lse) lse[static_cast<size_t>(h) * L.N + t] = (m + __log2f(wsum)) * 0.69314718055994531f;
+    if (lane == 0 && lse) lse[static_cast<size_t>(h) * L.Nl + t] = (m + __log2f(wsum)) * 0.69314718055994531f;
 }
 
 // Failure-path self-test: one thread waits on an mbarrier that nothing ever

@@ -16,6 +16,7 @@
 #include "plan.cuh"
 #include "score_kernel.cuh"
 #include "select_kernels.cuh"
+#include "shard_kernels.cuh"
 
 using namespace spava;
 
@@ -82,6 +83,10 @@ spava_status make_layer(const spava_config *c, Layer *L) {
         L->pcum[u + 1] = L->pcum[u] + std::min(L->l, n_u);
     }
     L->L = L->pcum[nc - 1];
+    // One GPU: every region held at its global position.
+    L->Nl = L->N;
+    L->own = nc >= 64 ? ~0ULL : ((1ULL << nc) - 1);
+    for (int r = 0; r < nc + 2; ++r) L->loc[r] = region_first(*L, r);
     const double scale = c->scale > 0.f ? static_cast<double>(c->scale) : 1.0 / std::sqrt(double(c->head_dim));
     L->scale_log2 = static_cast<float>(scale * 1.4426950408889634);
     return SPAVA_OK;
@@ -111,29 +116,38 @@ void region_rows(const Layer &L, int kind, int sub, int &lo, int &hi) {
 // tile descending, with the query heads of a KV head adjacent (shared K/V tiles
 // in L2; see decode_pair_item and decode_item).  Only regions lying inside
 // rows [row_lo, row_hi) are planned (the whole layer by default).
-int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int row_hi = INT32_MAX) {
+constexpr unsigned kAllKinds = (1u << kCtx) | (1u << kAnchor) | (1u << kQueryPart);
+int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int row_hi = INT32_MAX,
+                   unsigned kinds = kAllKinds) {
     struct G { Group g; int cost; };
     std::vector<G> gs;
     auto push = [&](int kind, int sub, int n_rt) {
         if (n_rt <= 0) return;
+        if (!stats && !((kinds >> kind) & 1u)) return;
         int lo, hi;
         region_rows(L, kind, sub, lo, hi);
         if (lo < row_lo || hi > row_hi) return;
         Item it{kind, sub, n_rt - 1, 0};
         gs.push_back({Group{kind, sub, n_rt, 0}, item_tiles(L, it)});
     };
+    // A query-row segment is computed where its keys are held: the anchor and
+    // the query block everywhere, chunk v where v is held.
+    auto seg_held = [&](int s) { return s == 0 || s > L.n_chunks || owns(L, s - 1); };
     const int n_qrt = cdiv(L.q, kRowTile);
     if (stats && L.norm == 0) {
-        for (int u = 0; u < L.n_chunks - 1; ++u) push(kStats, u, n_qrt);
+        for (int u = 0; u < L.n_chunks - 1; ++u)
+            if (owns(L, u)) push(kStats, u, n_qrt);
     } else if (stats) {
         // Row-normalised scores: the query rows' statistics over every segment
         // they attend (anchor, each chunk, the query block up to the row), the
         // same segments as the query-row partials of the attention.
         for (int s = (L.a > 0 ? 0 : 1); s < L.n_chunks + 2; ++s) push(kQueryPart, s, n_qrt);
     } else {
-        for (int v = 0; v < L.n_chunks; ++v) push(kCtx, v, cdiv(L.off[v + 1] - L.off[v], kRowTile));
+        for (int v = 0; v < L.n_chunks; ++v)
+            if (owns(L, v)) push(kCtx, v, cdiv(L.off[v + 1] - L.off[v], kRowTile));
         if (L.a > 0) push(kAnchor, 0, cdiv(L.a, kRowTile));
-        for (int s = (L.a > 0 ? 0 : 1); s < L.n_chunks + 2; ++s) push(kQueryPart, s, n_qrt);
+        for (int s = (L.a > 0 ? 0 : 1); s < L.n_chunks + 2; ++s)
+            if (seg_held(s)) push(kQueryPart, s, n_qrt);
     }
     std::stable_sort(gs.begin(), gs.end(), [](const G &x, const G &y) { return x.cost > y.cost; });
     // The statistics pass runs one row tile per CTA, the attention two.
@@ -231,9 +245,10 @@ spava_status encode_3d(CUtensorMap *tm, const void *base, uint64_t d0, uint64_t 
     return SPAVA_OK;
 }
 
-// Token-major [N, H, D] tensor, boxes of 64 columns x 1 head x 128 tokens.
+// Token-major [Nl, H, D] tensor (the rows held here), boxes of 64 columns x 1
+// head x 128 tokens.
 spava_status map_tokens(CUtensorMap *tm, const void *p, const Layer &L, int heads) {
-    return encode_3d(tm, p, L.d, heads, L.N, 64, 1, 128);
+    return encode_3d(tm, p, L.d, heads, L.Nl, 64, 1, 128);
 }
 // Packed [Hkv, rows, D] tensor, boxes of 64 columns x 128 rows x 1 head.
 spava_status map_packed(CUtensorMap *tm, const void *p, const Layer &L) {
@@ -319,7 +334,7 @@ spava_status run_scores(const Layer &L, const void *q, const void *k, float *sco
     int tiles = 0;
     for (int u = 0; u < L.n_chunks - 1; ++u) {
         p.tile_begin[u] = tiles;
-        tiles += cdiv(L.off[u + 1] - L.off[u], 128);
+        if (owns(L, u)) tiles += cdiv(L.off[u + 1] - L.off[u], 128);
     }
     p.tile_begin[L.n_chunks - 1] = tiles;
     const int64_t blocks = static_cast<int64_t>(tiles) * L.Hkv;
@@ -334,8 +349,15 @@ spava_status run_scores(const Layer &L, const void *q, const void *k, float *sco
     return launched();
 }
 
+// Producing chunks (u < 2H-1) held here.
+int owned_producers(const Layer &L) {
+    int n = 0;
+    for (int u = 0; u < L.n_chunks - 1; ++u) n += owns(L, u);
+    return n;
+}
+
 spava_status run_topk(const Layer &L, const float *scores, int32_t *idx, cudaStream_t st) {
-    const int blocks = (L.n_chunks - 1) * L.Hkv;
+    const int blocks = owned_producers(L) * L.Hkv;
     if (blocks == 0 || L.l == 0) return SPAVA_OK;
     topk_kernel<<<blocks, kSelectThreads, 0, st>>>(L, scores, idx);  // pools on the fly (L.pool)
     return launched();
@@ -367,23 +389,42 @@ spava_status run_pack(const Layer &L, const void *k, const void *v, const int32_
 // (producing chunk, KV head), then the anchor rows.
 spava_status run_select_pack(const Layer &L, const float *scores, int32_t *idx, const void *k,
                              const void *v, void *pk, void *pv, cudaStream_t st) {
-    const int64_t n_sel = static_cast<int64_t>(L.n_chunks - 1) * L.Hkv;
+    const int64_t n_sel = static_cast<int64_t>(owned_producers(L)) * L.Hkv;
     const int64_t n_anchor = L.a > 0 ? static_cast<int64_t>(L.Hkv) * cdiv(L.a, kAnchorRowsPerCta) : 0;
     const unsigned blocks = static_cast<unsigned>(n_sel + n_anchor);
+    if (blocks == 0) return SPAVA_OK;
     auto K = static_cast<const __nv_bfloat16 *>(k);
     auto V = static_cast<const __nv_bfloat16 *>(v);
     auto PK = static_cast<__nv_bfloat16 *>(pk);
     auto PV = static_cast<__nv_bfloat16 *>(pv);
     if (L.d == 128)
-        select_pack_kernel<128><<<blocks, kSelectThreads, 0, st>>>(L, scores, idx, K, V, PK, PV);
+        select_pack_kernel<128><<<blocks, kSelectThreads, 0, st>>>(L, scores, idx, K, V, PK, PV,
+                                                                   static_cast<int>(n_sel));
     else
-        select_pack_kernel<64><<<blocks, kSelectThreads, 0, st>>>(L, scores, idx, K, V, PK, PV);
+        select_pack_kernel<64><<<blocks, kSelectThreads, 0, st>>>(L, scores, idx, K, V, PK, PV,
+                                                                  static_cast<int>(n_sel));
+    return launched();
+}
+
+// The query rows: the per-segment partials merged by log-sum-exp.
+spava_status run_merge(const Layer &L, void *o, float *lse, char *ws, cudaStream_t st) {
+    const WsLayout w = ws_layout(L);
+    const float *part_O = reinterpret_cast<const float *>(ws + w.part_o);
+    const float *part_lse = reinterpret_cast<const float *>(ws + w.part_lse);
+    const int64_t warps = static_cast<int64_t>(L.Hq) * L.q;
+    const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
+    auto O = static_cast<__nv_bfloat16 *>(o);
+    if (L.d == 128)
+        merge_kernel<128><<<blocks, 256, 0, st>>>(L, part_O, part_lse, O, lse);
+    else
+        merge_kernel<64><<<blocks, 256, 0, st>>>(L, part_O, part_lse, O, lse);
     return launched();
 }
 
 spava_status run_attn(const Layer &L, const void *q, const void *k, const void *v, const void *pk,
                       const void *pv, void *o, float *lse, char *ws, cudaStream_t st,
-                      int row_lo = 0, int row_hi = INT32_MAX) {
+                      int row_lo = 0, int row_hi = INT32_MAX, unsigned kinds = kAllKinds,
+                      bool merge = true) {
     const WsLayout w = ws_layout(L);
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
@@ -394,7 +435,7 @@ spava_status run_attn(const Layer &L, const void *q, const void *k, const void *
     // With no packed rows (a = 0, l = 0) no segment reads the packed maps.
     SPAVA_TRY(L.L > 0 ? map_packed(&p.tmPK, pk, L) : map_tokens(&p.tmPK, k, L, L.Hkv));
     SPAVA_TRY(L.L > 0 ? map_packed(&p.tmPV, pv, L) : map_tokens(&p.tmPV, v, L, L.Hkv));
-    p.n_groups = plan_attention(L, false, p.groups, row_lo, row_hi);
+    p.n_groups = plan_attention(L, false, p.groups, row_lo, row_hi, kinds);
     p.O = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     p.part_O = reinterpret_cast<float *>(ws + w.part_o);
@@ -402,15 +443,8 @@ spava_status run_attn(const Layer &L, const void *q, const void *k, const void *
     p.status = reinterpret_cast<int *>(ws + w.status);
     p.queue = reinterpret_cast<int *>(ws + w.status + 128);  // inside the 256-byte status block
     SPAVA_TRY(L.d == 128 ? launch_attn<128, false>(p, st) : launch_attn<64, false>(p, st));
-    if (L.N - L.q < row_lo || L.N > row_hi) return SPAVA_OK;  // query block not in this range
-    const int64_t warps = static_cast<int64_t>(L.Hq) * L.q;
-    const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);
-    auto O = static_cast<__nv_bfloat16 *>(o);
-    if (L.d == 128)
-        merge_kernel<128><<<blocks, 256, 0, st>>>(L, p.part_O, p.part_lse, O, lse);
-    else
-        merge_kernel<64><<<blocks, 256, 0, st>>>(L, p.part_O, p.part_lse, O, lse);
-    return launched();
+    if (!merge || L.N - L.q < row_lo || L.N > row_hi) return SPAVA_OK;  // query block not in this range
+    return run_merge(L, o, lse, ws, st);
 }
 
 // Scoring, selection and gather: everything of the layer before the attention.
@@ -742,6 +776,297 @@ const char *spava_status_string(spava_status s) {
 }
 
 int32_t spava_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"
+
+// ==================================================================== shards
+// Multi-GPU ZigZag sequence parallelism ("Disposizione ZigZag", "Comunicazione
+// Sovrapposta"): `world` GPUs, rank r holding the physical hosts
+// p in [r*m, (r+1)*m), m = H / world, i.e. the chunks v with pair(v) / m == r,
+// in local buffers laid out [anchor | its chunks in increasing v | query].
+namespace {
+
+// The layer as rank `rank` of `world` sees it.
+spava_status make_shard_layer(const spava_config *c, int32_t rank, int32_t world, Layer *L) {
+    SPAVA_TRY(make_layer(c, L));
+    if (world < 1 || rank < 0 || rank >= world) return SPAVA_ERR_INVALID_ARG;
+    if (L->H % world) return SPAVA_ERR_UNSUPPORTED;
+    // Row-normalised scores need every chunk's statistics of the query rows
+    // before scoring, an exchange this path does not make.
+    if (L->norm) return SPAVA_ERR_UNSUPPORTED;
+    const int m = L->H / world, nc = L->n_chunks;
+    L->own = 0;
+    for (int v = 0; v < nc; ++v)
+        if (pair_of(L->H, v) / m == rank) L->own |= 1ULL << v;
+    for (int r = 0; r < nc + 2; ++r) L->loc[r] = -1;
+    int row = 0;
+    L->loc[0] = row;
+    row += L->a;
+    for (int v = 0; v < nc; ++v)
+        if (owns(*L, v)) {
+            L->loc[1 + v] = row;
+            row += L->off[v + 1] - L->off[v];
+        }
+    L->loc[nc + 1] = row;
+    L->Nl = row + L->q;
+    return SPAVA_OK;
+}
+
+// Chunks of rank r (ascending): the slots of its exchange messages.
+int shard_chunks(const Layer &L, int world, int r, int *out) {
+    const int m = L.H / world;
+    int n = 0;
+    for (int v = 0; v < L.n_chunks; ++v)
+        if (pair_of(L.H, v) / m == r) out[n++] = v;
+    return n;
+}
+
+// Passing-block message of one rank: per slot (one of its 2m chunks) the
+// indices [Hkv, l] int32, then K rows [Hkv, l, d] and V rows [Hkv, l, d] bf16;
+// the slot of the last chunk (no successor) stays unused.
+struct PassMsg { size_t idx, k, v, total; };
+PassMsg pass_msg(const Layer &L, int world) {
+    const size_t slots = 2 * (L.H / world);
+    PassMsg g{};
+    size_t o = 0;
+    auto take = [&](size_t b) { size_t at = o; o = align256(o + b); return at; };
+    g.idx = take(slots * L.Hkv * L.l * 4);
+    g.k = take(slots * L.Hkv * L.l * L.d * 2);
+    g.v = take(slots * L.Hkv * L.l * L.d * 2);
+    g.total = std::max<size_t>(o, 256);
+    return g;
+}
+
+// Query-partial message of one rank: per slot the normalised partial O
+// [Hq, q, d] and the base-2 lse [Hq, q] of the query rows over that chunk.
+struct PartMsg { size_t o, lse, total; };
+PartMsg part_msg(const Layer &L, int world) {
+    const size_t slots = 2 * (L.H / world);
+    PartMsg g{};
+    size_t o = 0;
+    auto take = [&](size_t b) { size_t at = o; o = align256(o + b); return at; };
+    g.o = take(slots * L.Hq * L.q * L.d * 4);
+    g.lse = take(slots * L.Hq * L.q * 4);
+    g.total = o;
+    return g;
+}
+
+// Collects 2-D copies and launches them, kMaxCopyJobs per launch.
+struct Copier {
+    CopyBatch b{};
+    int64_t most = 0;  // units of the largest job of the batch
+    cudaStream_t st;
+    explicit Copier(cudaStream_t s) : st(s) {}
+    spava_status add(const void *src, int64_t src_pitch, void *dst, int64_t dst_pitch, int64_t width,
+                     int64_t height) {
+        if (width <= 0 || height <= 0) return SPAVA_OK;
+        const auto a = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) |
+                       static_cast<uintptr_t>(src_pitch) | static_cast<uintptr_t>(dst_pitch) |
+                       static_cast<uintptr_t>(width);
+        const int unit = (a & 15) == 0 ? 16 : 4;
+        if (a & 3) return SPAVA_ERR_MISALIGNED;
+        if (width >= (1LL << 31) || height >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
+        if (b.n == kMaxCopyJobs) SPAVA_TRY(flush());
+        b.job[b.n++] = CopyJob{static_cast<const char *>(src), static_cast<char *>(dst), src_pitch,
+                               dst_pitch, static_cast<int32_t>(width), static_cast<int32_t>(height),
+                               unit, 0};
+        most = std::max(most, width / unit * height);
+        return SPAVA_OK;
+    }
+    spava_status flush() {
+        if (b.n == 0) return SPAVA_OK;
+        const int64_t blocks = std::min<int64_t>((most + 255) / 256, 1024);
+        batched_copy_kernel<<<dim3(static_cast<unsigned>(blocks), static_cast<unsigned>(b.n)), 256, 0, st>>>(b);
+        b.n = 0;
+        most = 0;
+        return launched();
+    }
+};
+
+// Copies between the workspace's passing blocks (idx [2H-1, Hkv, l], packed
+// K/V [Hkv, L, d]) and slot k of a pass message: to_msg = export.
+spava_status pass_slot_copy(Copier &cp, const Layer &L, char *ws, char *msg, const PassMsg &g, int k,
+                            int u, bool to_msg) {
+    if (u >= L.n_chunks - 1 || L.l == 0) return SPAVA_OK;  // no passing block
+    const WsLayout w = ws_layout(L);
+    const int64_t l_eff = std::min(L.l, L.off[u + 1] - L.off[u]);
+    const int64_t row = int64_t(L.d) * 2;
+    char *idx_ws = ws + w.idx + size_t(u) * L.Hkv * L.l * 4;
+    char *idx_m = msg + g.idx + size_t(k) * L.Hkv * L.l * 4;
+    const int64_t idx_bytes = int64_t(L.Hkv) * L.l * 4;
+    if (to_msg) SPAVA_TRY(cp.add(idx_ws, idx_bytes, idx_m, idx_bytes, idx_bytes, 1));
+    else SPAVA_TRY(cp.add(idx_m, idx_bytes, idx_ws, idx_bytes, idx_bytes, 1));
+    for (int kv = 0; kv < 2; ++kv) {
+        char *packed = ws + (kv ? w.pv : w.pk) + size_t(L.pcum[u]) * row;     // KV head 0
+        char *slot = msg + (kv ? g.v : g.k) + size_t(k) * L.Hkv * L.l * row;  // KV head 0
+        const int64_t packed_pitch = int64_t(L.L) * row, slot_pitch = int64_t(L.l) * row;
+        if (to_msg) SPAVA_TRY(cp.add(packed, packed_pitch, slot, slot_pitch, l_eff * row, L.Hkv));
+        else SPAVA_TRY(cp.add(slot, slot_pitch, packed, packed_pitch, l_eff * row, L.Hkv));
+    }
+    return SPAVA_OK;
+}
+
+// Copies between the workspace's query partials of segment 1+v and slot k of
+// a partial message.
+spava_status part_slot_copy(Copier &cp, const Layer &L, char *ws, char *msg, const PartMsg &g, int k,
+                            int v, bool to_msg) {
+    const WsLayout w = ws_layout(L);
+    const int64_t o_bytes = int64_t(L.Hq) * L.q * L.d * 4, l_bytes = int64_t(L.Hq) * L.q * 4;
+    char *o_ws = ws + w.part_o + size_t(1 + v) * o_bytes, *o_m = msg + g.o + size_t(k) * o_bytes;
+    char *l_ws = ws + w.part_lse + size_t(1 + v) * l_bytes, *l_m = msg + g.lse + size_t(k) * l_bytes;
+    // Rows of d floats (o) and one row of Hq*q floats (lse).
+    const int64_t o_row = int64_t(L.d) * 4, o_rows = int64_t(L.Hq) * L.q;
+    if (to_msg) {
+        SPAVA_TRY(cp.add(o_ws, o_row, o_m, o_row, o_row, o_rows));
+        SPAVA_TRY(cp.add(l_ws, l_bytes, l_m, l_bytes, l_bytes, 1));
+    } else {
+        SPAVA_TRY(cp.add(o_m, o_row, o_ws, o_row, o_row, o_rows));
+        SPAVA_TRY(cp.add(l_m, l_bytes, l_ws, l_bytes, l_bytes, 1));
+    }
+    return SPAVA_OK;
+}
+
+spava_status check_shard_args(const Layer &L, void *ws, size_t ws_bytes) {
+    return check_ws(L, ws, ws_bytes);
+}
+
+}  // namespace
+
+extern "C" {
+
+spava_status spava_shard_layout(const spava_config *cfg, int32_t rank, int32_t world,
+                                int64_t *local_first, int64_t *n_local, int32_t *slot_chunk) {
+    Layer L;
+    SPAVA_TRY(make_shard_layer(cfg, rank, world, &L));
+    if (local_first)
+        for (int r = 0; r < L.n_chunks + 2; ++r) local_first[r] = L.loc[r];
+    if (n_local) *n_local = L.Nl;
+    if (slot_chunk) {
+        int ch[kMaxChunks];
+        const int n = shard_chunks(L, world, rank, ch);
+        for (int k = 0; k < n; ++k) slot_chunk[k] = ch[k];
+    }
+    return SPAVA_OK;
+}
+
+spava_status spava_shard_sizes(const spava_config *cfg, int32_t world, size_t *ws_bytes,
+                               size_t *pass_msg_bytes, size_t *part_msg_bytes) {
+    Layer L;
+    SPAVA_TRY(make_shard_layer(cfg, 0, world, &L));
+    if (ws_bytes) *ws_bytes = ws_layout(L).total;
+    if (pass_msg_bytes) *pass_msg_bytes = pass_msg(L, world).total;
+    if (part_msg_bytes) *part_msg_bytes = part_msg(L, world).total;
+    return SPAVA_OK;
+}
+
+spava_status spava_shard_front(const spava_config *cfg, int32_t rank, int32_t world, const void *q,
+                               const void *k, const void *v, void *pass_send, void *ws,
+                               size_t ws_bytes, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_shard_layer(cfg, rank, world, &L));
+    SPAVA_TRY(check_ptr(q));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(v));
+    SPAVA_TRY(check_ptr(pass_send));
+    SPAVA_TRY(check_shard_args(L, ws, ws_bytes));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(ws);
+    SPAVA_TRY(run_front(L, q, k, v, nullptr, w, st));
+    const PassMsg g = pass_msg(L, world);
+    int ch[kMaxChunks];
+    const int n = shard_chunks(L, world, rank, ch);
+    Copier cp(st);
+    for (int s = 0; s < n; ++s)
+        SPAVA_TRY(pass_slot_copy(cp, L, w, static_cast<char *>(pass_send), g, s, ch[s], true));
+    return cp.flush();
+}
+
+spava_status spava_shard_local_attn(const spava_config *cfg, int32_t rank, int32_t world,
+                                    const void *q, const void *k, const void *v, void *o, float *lse,
+                                    void *part_send, void *ws, size_t ws_bytes, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_shard_layer(cfg, rank, world, &L));
+    SPAVA_TRY(check_ptr(q));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(v));
+    SPAVA_TRY(check_ptr(o));
+    SPAVA_TRY(check_ptr(lse, false));
+    SPAVA_TRY(check_ptr(part_send));
+    SPAVA_TRY(check_shard_args(L, ws, ws_bytes));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(ws);
+    const WsLayout lay = ws_layout(L);
+    // Anchor rows and the query rows' partials over the anchor, this rank's
+    // chunks and the query block: nothing from another rank is needed.
+    SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st, 0, INT32_MAX,
+                       (1u << kAnchor) | (1u << kQueryPart), false));
+    const PartMsg g = part_msg(L, world);
+    int ch[kMaxChunks];
+    const int n = shard_chunks(L, world, rank, ch);
+    Copier cp(st);
+    for (int s = 0; s < n; ++s)
+        SPAVA_TRY(part_slot_copy(cp, L, w, static_cast<char *>(part_send), g, s, ch[s], true));
+    return cp.flush();
+}
+
+spava_status spava_shard_context_attn(const spava_config *cfg, int32_t rank, int32_t world,
+                                      const void *q, const void *k, const void *v,
+                                      const void *pass_all, void *o, float *lse, int32_t *idx_out,
+                                      void *ws, size_t ws_bytes, void *stream) {
+    Layer L;
+    SPAVA_TRY(make_shard_layer(cfg, rank, world, &L));
+    SPAVA_TRY(check_ptr(q));
+    SPAVA_TRY(check_ptr(k));
+    SPAVA_TRY(check_ptr(v));
+    SPAVA_TRY(check_ptr(o));
+    SPAVA_TRY(check_ptr(lse, false));
+    SPAVA_TRY(check_ptr(pass_all));
+    SPAVA_TRY(check_ptr(idx_out, false));
+    SPAVA_TRY(check_shard_args(L, ws, ws_bytes));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(ws);
+    const WsLayout lay = ws_layout(L);
+    const PassMsg g = pass_msg(L, world);
+    // Every other rank's passing blocks into the packed buffer.
+    Copier cp(st);
+    for (int r = 0; r < world; ++r) {
+        if (r == rank) continue;
+        int ch[kMaxChunks];
+        const int n = shard_chunks(L, world, r, ch);
+        char *msg = const_cast<char *>(static_cast<const char *>(pass_all)) + size_t(r) * g.total;
+        for (int s = 0; s < n; ++s) SPAVA_TRY(pass_slot_copy(cp, L, w, msg, g, s, ch[s], false));
+    }
+    if (idx_out && L.l > 0) {
+        const int64_t b = int64_t(L.n_chunks - 1) * L.Hkv * L.l * 4;
+        SPAVA_TRY(cp.add(w + lay.idx, b, idx_out, b, b, 1));
+    }
+    SPAVA_TRY(cp.flush());
+    return run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st, 0, INT32_MAX, 1u << kCtx, false);
+}
+
+spava_status spava_shard_merge(const spava_config *cfg, int32_t rank, int32_t world,
+                               const void *part_all, void *o, float *lse, void *ws, size_t ws_bytes,
+                               void *stream) {
+    Layer L;
+    SPAVA_TRY(make_shard_layer(cfg, rank, world, &L));
+    SPAVA_TRY(check_ptr(o));
+    SPAVA_TRY(check_ptr(lse, false));
+    SPAVA_TRY(check_ptr(part_all));
+    SPAVA_TRY(check_shard_args(L, ws, ws_bytes));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(ws);
+    const PartMsg g = part_msg(L, world);
+    Copier cp(st);
+    for (int r = 0; r < world; ++r) {
+        if (r == rank) continue;
+        int ch[kMaxChunks];
+        const int n = shard_chunks(L, world, r, ch);
+        char *msg = const_cast<char *>(static_cast<const char *>(part_all)) + size_t(r) * g.total;
+        for (int s = 0; s < n; ++s) SPAVA_TRY(part_slot_copy(cp, L, w, msg, g, s, ch[s], false));
+    }
+    SPAVA_TRY(cp.flush());
+    return run_merge(L, o, lse, w, st);
+}
 
 }  // extern "C"
 

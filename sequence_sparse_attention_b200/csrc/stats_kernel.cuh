@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(kStatsThreads, 1) stats_kernel(const __grid_co
     int row0, row_end;
     item_rows(L, it, row0, row_end);
     const int g = it.h / L.G;
+    const int rs = region_shift(L, item_region(L, it));  // global minus local row of the Q rows
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(kStatsThreads, 1) stats_kernel(const __grid_co
         if (lane == 0) {
             mbar_expect_tx(q_full, SM::kTile);
             for (int p = 0; p < SM::kPanels; ++p)
-                tma_load_3d(smem + SM::kOffQ + p * 16384, &P.tmQ, p * 64, it.h, row0, q_full);
+                tma_load_3d(smem + SM::kOffQ + p * 16384, &P.tmQ, p * 64, it.h, row0 - rs, q_full);
             int k_last[KS];
             for (int i = 0; i < KS; ++i) k_last[i] = -1;
             TileCursor kc;
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kStatsThreads, 1) stats_kernel(const __grid_co
                 const Seg &s = segs[kc.seg];
                 const int key0 = s.begin + kc.tile * kKeyTile;
                 for (int p = 0; p < SM::kPanels; ++p)
-                    tma_load_3d(kd + p * 16384, &P.tmK, p * 64, g, key0, &k_full[ks]);
+                    tma_load_3d(kd + p * 16384, &P.tmK, p * 64, g, key0 - s.shift, &k_full[ks]);
                 k_last[ks] = j;
                 kc.advance(segs);
             }

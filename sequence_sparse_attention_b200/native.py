@@ -21,7 +21,9 @@ EXPORTS = ("spava_workspace_size", "spava_packed_len", "spava_score", "spava_top
            "spava_pack_passing", "spava_attn", "spava_prefill_attention",
            "spava_prefill_attention_host", "spava_device_status", "spava_attended_pairs",
            "spava_status_string", "spava_last_cuda_error", "spava_score_noalloc",
-           "spava_selftest_wait_timeout", "spava_plan_chunks", "spava_score_noalloc_status")
+           "spava_selftest_wait_timeout", "spava_plan_chunks", "spava_score_noalloc_status",
+           "spava_shard_layout", "spava_shard_sizes", "spava_shard_front", "spava_shard_local_attn",
+           "spava_shard_context_attn", "spava_shard_merge")
 
 
 class SpavaConfig(ctypes.Structure):
@@ -63,6 +65,7 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     vp, sz, cfgp = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(SpavaConfig)
     i64p = ctypes.POINTER(ctypes.c_int64)
+    i32, szp = ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)
     sig = {
         "spava_workspace_size": [cfgp, ctypes.POINTER(ctypes.c_size_t)],
         "spava_packed_len": [cfgp, i64p],
@@ -78,6 +81,12 @@ def load() -> ctypes.CDLL:
         "spava_score_noalloc_status": [vp, ctypes.POINTER(ctypes.c_int32)],
         "spava_selftest_wait_timeout": [vp, sz, vp],
         "spava_plan_chunks": [ctypes.c_int32, i64p, ctypes.c_int64, ctypes.c_int64, i64p],
+        "spava_shard_layout": [cfgp, i32, i32, i64p, i64p, ctypes.POINTER(ctypes.c_int32)],
+        "spava_shard_sizes": [cfgp, i32, szp, szp, szp],
+        "spava_shard_front": [cfgp, i32, i32, vp, vp, vp, vp, vp, sz, vp],
+        "spava_shard_local_attn": [cfgp, i32, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "spava_shard_context_attn": [cfgp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "spava_shard_merge": [cfgp, i32, i32, vp, vp, vp, vp, sz, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
