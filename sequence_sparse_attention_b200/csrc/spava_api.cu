@@ -851,7 +851,9 @@ PartMsg part_msg(const Layer &L, int world) {
     return g;
 }
 
-// Collects 2-D copies and launches them, kMaxCopyJobs per launch.
+// Collects 2-D copies and launches them, kMaxCopyJobs per launch.  The jobs
+// of one launch run concurrently: none may read what another writes (flush
+// between dependent copies).
 struct Copier {
     CopyBatch b{};
     int64_t most = 0;  // units of the largest job of the batch
@@ -1036,11 +1038,12 @@ spava_status spava_shard_context_attn(const spava_config *cfg, int32_t rank, int
         char *msg = const_cast<char *>(static_cast<const char *>(pass_all)) + size_t(r) * g.total;
         for (int s = 0; s < n; ++s) SPAVA_TRY(pass_slot_copy(cp, L, w, msg, g, s, ch[s], false));
     }
-    if (idx_out && L.l > 0) {
+    SPAVA_TRY(cp.flush());
+    if (idx_out && L.l > 0) {  // after the imports that complete the indices
         const int64_t b = int64_t(L.n_chunks - 1) * L.Hkv * L.l * 4;
         SPAVA_TRY(cp.add(w + lay.idx, b, idx_out, b, b, 1));
+        SPAVA_TRY(cp.flush());
     }
-    SPAVA_TRY(cp.flush());
     return run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st, 0, INT32_MAX, 1u << kCtx, false);
 }
 
