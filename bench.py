@@ -12,9 +12,11 @@ A second timed region runs the same layer as the four separate C-ABI steps
 CUDA events between them, for the per-kernel split and the roofline of the
 attention launch.  Prints one JSON line (rank 0).
 
-Multi-GPU: each rank runs its own independent layer (weak scaling, no data
-collective); the process group only provides the barrier and the max-over-ranks
-timing.  ``--impl reference`` times the fp64 CPU oracle on a bounded sample of
+Multi-GPU (torchrun, N > 1): the one layer is split over the ranks by the
+ZigZag sequence parallelism (rank r holds physical hosts r*H/N .. (r+1)*H/N-1,
+i.e. chunk pairs p and 2H-1-p), with NCCL all-gathers of the passing blocks
+and the query partials -- strong scaling of the layer; the time is the
+slowest rank's.  ``--impl reference`` times the fp64 CPU oracle on a bounded sample of
 the same workload instead (rank 0 only).
 """
 from __future__ import annotations
@@ -159,11 +161,12 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
-def job_throughput(tokens_per_rank: int, steps: int, ms_rank: float, world: int) -> tuple:
-    """Whole-job tokens/s: every rank processes its own layer (weak scaling); the
-    elapsed time is the slowest rank's.  Returns (tokens/s, ms per step)."""
+def job_throughput(tokens_per_step: int, steps: int, ms_rank: float, world: int) -> tuple:
+    """Whole-job tokens/s: the layer's tokens per step, all ranks together (the
+    ranks share one layer: strong scaling); the elapsed time is the slowest
+    rank's.  Returns (tokens/s, ms per step)."""
     ms = max_over_ranks(ms_rank, world)
-    return world * tokens_per_rank * steps / (ms / 1e3), ms / steps
+    return tokens_per_step * steps / (ms / 1e3), ms / steps
 
 
 def barrier(world: int):
@@ -253,7 +256,7 @@ def run_reference(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * w.N / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
+        "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -261,8 +264,14 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w):
-    return {"workload": f"{w.name}: H={w.H} ({2 * w.H} ZigZag virtual hosts), {w.Hq} q / {w.Hkv} kv heads, "
+def parallelism(world: int) -> str:
+    return ("one GPU, all 2H ZigZag virtual hosts on it" if world == 1 else
+            f"ZigZag sequence parallelism over {world} GPUs (H/{world} physical hosts each; "
+            "NCCL all-gathers of passing blocks and query partials)")
+
+
+def workload_config(w, world=1):
+    return {"parallelism": parallelism(world),"workload": f"{w.name}: H={w.H} ({2 * w.H} ZigZag virtual hosts), {w.Hq} q / {w.Hkv} kv heads, "
                         f"d={w.d}, {w.N} tokens (anchor {w.a}, query block {w.q}), top-l={w.l}",
             "tokens": w.N, "H": w.H, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
             "anchor": w.a, "query_block": w.q, "top_l": w.l,
@@ -437,7 +446,7 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic", "config": workload_config(w, world),
         "roofline": roofline,
         "selection_hbm": selection,
         "kernel_ms": per,
@@ -455,6 +464,134 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def run_sharded(args, world, rank, local):
+    """N > 1: the one layer split over the ranks (ZigZag sequence parallelism).
+    Each rank holds [anchor | its chunks | query block]; the passing blocks and
+    the query partials are NCCL all-gathers on a second stream, overlapped with
+    the rank's local attention.  ``--shard-on-one`` runs this path as world 1
+    (the gathers are copies) to check it on a single GPU."""
+    from sequence_sparse_attention_b200.api import Layout, SpavaShard, attended_pairs
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = selected_workload(args)
+    lay = Layout.from_workload(w)
+    sh = SpavaShard(lay, rank, world, device)
+    Q, K, V, off = make_inputs(w, device)
+    pos = torch.from_numpy(sh.positions).to(device)
+    q, k, v = Q[pos].contiguous(), K[pos].contiguous(), V[pos].contiguous()
+    del Q, K, V
+    torch.cuda.empty_cache()
+    o, lse = sh.new_outputs()
+    if world > 1:
+        import torch.distributed as dist
+
+        def all_gather(out, inp):
+            dist.all_gather_into_tensor(out, inp)
+    else:
+        def all_gather(out, inp):
+            out.copy_(inp)
+    cs = torch.cuda.Stream(device)
+
+    def layer():
+        sh.layer(q, k, v, o, lse, all_gather, comm_stream=cs)
+
+    for _ in range(args.warmup):
+        layer()
+    torch.cuda.synchronize()
+    if int(sh.ws[:4].view(torch.int32).item()):
+        raise RuntimeError("kernel status set during warm-up")
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_ev = 5
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    sampler = ClockSampler(physical_gpu(local))
+    with sampler:
+        time.sleep(0.3)
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record()
+        for _ in range(args.steps):
+            layer()
+        end.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        # per-call split on the compute stream, the gathers done in place
+        for s_ in range(args.steps):
+            ev = evs[s_]
+            ev[0].record()
+            sh.front(q, k, v)
+            ev[1].record()
+            sh.local_attn(q, k, v, o, lse)
+            all_gather(sh.pass_all, sh.pass_send)
+            all_gather(sh.part_all, sh.part_send)
+            ev[2].record()
+            sh.context_attn(q, k, v, o, lse)
+            ev[3].record()
+            sh.merge(o, lse)
+            ev[4].record()
+        torch.cuda.synchronize()
+        barrier(world)
+    clocks = sampler.summary()
+    if int(sh.ws[:4].view(torch.int32).item()):
+        raise RuntimeError("kernel status set during the timed region")
+    tokens_per_s, ms_step = job_throughput(w.N, args.steps, start.elapsed_time(end), world)
+    names = ["front", "local_attn_and_gathers", "context_attn", "merge"]
+    per = {n: statistics.mean(evs[s_][i].elapsed_time(evs[s_][i + 1]) for s_ in range(args.steps))
+           for i, n in enumerate(names)}
+
+    # roofline: the context-row attention launch of this rank
+    pk_, pe = peaks()
+    _, per_host = attended_pairs(lay)
+    m = w.H // world
+    ctx_pairs = sum(per_host[rank * m:(rank + 1) * m])
+    flops = 4.0 * w.d * w.Hq * ctx_pairs
+    achieved = flops / (per["context_attn"] / 1e3) / 1e12
+    peak = pk_.get("bf16_tflops")
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "attn_kernel<128>, context rows of this rank's chunks (spava_shard_context_attn)",
+                "peak_kind": f"{pe} bf16 dense GEMM, burst", "rank": rank,
+                "algorithmic_flops_per_launch": flops}
+
+    # end to end: pinned host buffers of this rank's rows in, its O rows out
+    qh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    kh = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+    vh = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+    qh.copy_(q)
+    kh.copy_(k)
+    vh.copy_(v)
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        layer()
+        oh.copy_(o, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    e2e = {"value": w.N / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * 2,
+           "d2h_bytes_per_step": o.numel() * 2, "ms_per_step": e2e_ms,
+           "api": "SpavaShard.layer per rank: pinned host copies of the rank's rows in, its O rows out"}
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(w, world),
+        "roofline": roofline, "kernel_ms_rank": per, "e2e": e2e,
+        "gpu_launches": args.steps * 10, "clocks": clocks,
+        "messages_bytes": {"pass_per_rank": sh.pass_send.numel(), "part_per_rank": sh.part_send.numel()},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -468,6 +605,8 @@ def main():
                     help="selection variant: 1 = row-normalised scores")
     ap.add_argument("--score-pool", type=int, default=0,
                     help="selection variant: odd window w >= 3 = pooled ranking")
+    ap.add_argument("--shard-on-one", action="store_true",
+                    help="run the sharded (multi-GPU) path as one rank")
     args = ap.parse_args()
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -475,7 +614,10 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_ours(args, world, rank, local)
+        if world > 1 or args.shard_on_one:
+            run_sharded(args, world, rank, local)
+        else:
+            run_ours(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

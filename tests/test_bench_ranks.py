@@ -1,6 +1,6 @@
 """bench.py's multi-rank timing on CPU: two gloo ranks, each with its own
 elapsed time; the job's time is the slowest rank's and the throughput counts
-every rank's tokens (independent layers per GPU, weak scaling)."""
+the layer's tokens once (the ranks share one layer: strong scaling)."""
 import os
 import socket
 
@@ -42,4 +42,4 @@ def test_two_gloo_ranks_take_the_slowest_time():
     for rank, mx, tps, ms_step in res:
         assert mx == 1.0
         assert ms_step == pytest.approx(50.0)
-        assert tps == pytest.approx(2 * 131072 * 10 / 0.5)
+        assert tps == pytest.approx(131072 * 10 / 0.5)
