@@ -29,6 +29,14 @@
 // The commit that announces S_X(j+1) tracks every earlier MMA of the thread,
 // PV_X(j) included, so whenever the softmax of tile X sees a new S, O_X is
 // stable and can be rescaled without a further wait.
+//
+// STATS = true is the statistics pass of the scoring ("Blocchi di Passaggio":
+// each chunk's keys are scored by the query block's softmax over that chunk):
+// the same key tiles, max and sum in the same order, but no V, no PV and no P;
+// the item's per-row base-2 log-sum-exp goes to P.stats.  The running sum is
+// the very arithmetic of the full kernel, so the statistics equal, bit for
+// bit, the log-sum-exps the full kernel's query-row partials carry -- the
+// scoring may take either.
 #pragma once
 
 #include "plan.cuh"
@@ -45,7 +53,7 @@ struct AttnParams {
     float *lse;         // [Hq, N] natural log, or null
     float *part_O;      // [2H+2, Hq, q, D] normalised partials of the query rows
     float *part_lse;    // [2H+2, Hq, q] log2 domain
-    float *stats;       // [2H-1, Hq, q] log2-domain lse of the query rows per chunk
+    float *stats;       // STATS: [segments, Hq, q] log2-domain lse of the query rows
     int *status;        // workspace status word
     int *queue;         // work-item counter of the persistent attention grid (zeroed per launch)
     int32_t n_items;    // work items of the attention launch
@@ -189,7 +197,7 @@ __device__ __forceinline__ void plan_item(const Layer &L, const Group *groups, i
     ip.TB = ip.hasB ? ip.T : 0;
 }
 
-template <int D>
+template <int D, bool STATS = false>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_constant__ AttnParams P) {
     using SM = AttnSmem<D>;
     constexpr int KS = SM::KS, VS = SM::VS;
@@ -342,7 +350,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
             bool live = T > 0 ? load_k(0) : true;
             for (int j = 0; live && j < T; ++j) {
                 if (j + 1 < T) live = load_k(j + 1);
-                if (live) live = load_v(j);
+                if (!STATS && live) live = load_v(j);
             }
             // Every load this thread issued has landed before the CTA may exit.
             mbar_wait_drain(q_full, 0);
@@ -397,7 +405,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 if (TB > 0) mma_s(1, 0);
                 tc_commit(&k_empty[0]);
             }
-            for (int j = 0; ok && j < T; ++j) {
+            // Statistics only: S_X(j+1) as soon as the softmax has read S_X(j).
+            for (int j = 0; STATS && ok && j < T; ++j) {
+                const int kn = j + 1, ks = kn % KS;
+                bool k_seen = false;
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const int TX = x ? TB : TA;
+                    if (ok && j < TX) {
+                        ok = mbar_wait(&p_full[x], j & 1, ab);
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (kn < TX) {
+                            if (!k_seen) {
+                                ok = mbar_wait(&k_full[ks], (kn / KS) & 1, ab);
+                                if (!ok) break;
+                                tc_fence_after();
+                                k_seen = true;
+                            }
+                            mma_s(x, kn);
+                        }
+                    }
+                }
+                if (!ok) break;
+                if (k_seen) tc_commit(&k_empty[ks]);
+            }
+            for (int j = 0; !STATS && ok && j < T; ++j) {
                 const int vs = j % VS, kn = j + 1, ks = kn % KS;
                 if (!mbar_wait(&v_full[vs], (j / VS) & 1, ab)) break;
                 bool k_seen = false;
@@ -481,21 +514,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                     for (int e = 0; e < 32; ++e) xs[c * 32 + e] = __uint_as_float(u[c][e]);
                 }
             }
+            if (STATS) {  // S_X(j) is in registers: the next S may overwrite it
+                tc_fence_before();
+                mbar_arrive(&p_full[x]);
+            }
             if (lim < kKeyTile) {  // only tiles crossing a segment end or the diagonal
 #pragma unroll
                 for (int c = 0; c < kKeyTile; ++c)
                     if (c >= lim) xs[c] = -INFINITY;
             }
-            const float mx = max128(xs) * sl2;
+            // Rounded operations (never contracted into FMAs), so that the
+            // statistics pass repeats this arithmetic exactly.
+            const float mx = __fmul_rn(max128(xs), sl2);
             const float m_new = fmaxf(m_run, mx);
             const bool need = m_new > m_run + 8.0f;
             float alpha = 1.f;
             if (need) {
-                alpha = ex2(m_run - m_new);
-                l_run *= alpha;
+                alpha = ex2(__fsub_rn(m_run, m_new));
+                l_run = __fmul_rn(l_run, alpha);
                 m_run = m_new;
             }
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
+            if (!STATS && j > 0 && __any_sync(0xffffffffu, need)) {
                 // O_X holds the sum up to tile j-1 scaled by the old max, and is
                 // stable: PV_X(j-1) completed before S_X(j) was announced.
 #pragma unroll 1
@@ -524,25 +563,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                     const float2 arg = ffma2(make_float2(xs[c * 32 + 2 * e], xs[c * 32 + 2 * e + 1]), sl2v, nmu);
                     const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
                     ps[e & 1] = fadd2(ps[e & 1], p);
-                    pk[e] = pack_bf16x2(p.x, p.y);
+                    if (!STATS) pk[e] = pack_bf16x2(p.x, p.y);
                 }
-                tmem_st16(lane_addr + col_s + c * 16, pk);
+                if (!STATS) tmem_st16(lane_addr + col_s + c * 16, pk);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&p_full[x]);
+            if (!STATS) {
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&p_full[x]);
+            }
             const float2 pss = fadd2(ps[0], ps[1]);
-            l_run += pss.x + pss.y;
+            l_run = __fadd_rn(l_run, __fadd_rn(pss.x, pss.y));
         }
 
         // ------------------------------------------------------------ epilogue
-        if (ok && TX > 0) {
+        if (STATS) {
+            // The row's base-2 log-sum-exp over the item's keys.
+            if (ok && t < row_end) {
+                const int i = t - (L.N - L.q);
+                P.stats[(static_cast<size_t>(it.sub) * L.Hq + hx) * L.q + i] =
+                    (l_run > 0.f) ? __fadd_rn(m_run, __log2f(l_run)) : -INFINITY;
+            }
+        } else if (ok && TX > 0) {
             ok = __all_sync(0xffffffffu, mbar_wait(&o_done[x], 0, ab));
             if (ok) {
                 tc_fence_after();
                 const bool valid = t < row_end;
                 const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-                const float lse2 = (l_run > 0.f) ? m_run + __log2f(l_run) : -INFINITY;
+                const float lse2 = (l_run > 0.f) ? __fadd_rn(m_run, __log2f(l_run)) : -INFINITY;
                 if (it.kind == kQueryPart) {
                     const int i = t - (L.N - L.q);
                     float *dst = P.part_O + ((static_cast<size_t>(it.sub) * L.Hq + hx) * L.q + i) * D;

@@ -5,18 +5,27 @@
 // scores.  Score of key j of chunk u for KV head g:
 //     S[g, j] = sum_{h in g} sum_{i in query block} exp2(x_{h,i,j} - lse2_{u,h,i}),
 //     x = scale*log2(e) * q_{h,i} . k_{g,j},
-// where lse2_{u,h,i} is the base-2 log-sum-exp of row (h, i) over chunk u (the
-// statistics pass, stats_kernel.cuh).  Equivalently: softmax over the
-// chunk, summed over query rows and group heads.
+// where lse2_{u,h,i} is the base-2 log-sum-exp of row (h, i) over chunk u:
+// from the attention kernel's statistics mode, or -- the same values -- from
+// the query-row partial of chunk u ("Forward Fuso di Contesto e Query").
+// Equivalently: softmax over the chunk, summed over query rows and group heads.
 //
 // One CTA = 128 keys of one chunk and one KV head.  The product is formed
 // transposed, S^T = K Q^T (M = 128 keys, N = 128 query rows of one head per
 // block, K = d), so that TMEM lane j holds key j and each thread sums its own
 // key's probabilities without any cross-thread reduction; the summation order
 // is fixed, so the result is deterministic.
+//
+// FUSED = true also selects and gathers (the layer entry points): the CTA that
+// writes the last 128-key tile of a (chunk, KV head) -- counted with an atomic
+// per (chunk, KV head) -- selects that chunk's passing block for the KV head
+// (select_chunk) and copies its K/V rows into the packed buffer; the CTAs after
+// the scoring ones copy the anchor rows.  Selections of finished chunks thus
+// run while later chunks are still being scored.
 #pragma once
 
 #include "plan.cuh"
+#include "select_kernels.cuh"
 #include "sm100.cuh"
 
 namespace spava {
@@ -28,6 +37,12 @@ struct ScoreParams {
     float *scores;       // [Hkv, C]
     int *status;
     int32_t tile_begin[kMaxChunks + 1];  // prefix of 128-key tiles over chunks u < 2H-1
+    // FUSED only
+    int *counters;       // [2H-1, Hkv] finished tiles, zero at launch
+    int32_t *idx;        // [2H-1, Hkv, l]
+    const __nv_bfloat16 *K, *V;
+    __nv_bfloat16 *PK, *PV;  // [Hkv, L, D]
+    int32_t n_score_ctas;
 };
 
 constexpr int kScoreWarps = 16;                 // 4 per TMEM lane quarter
@@ -54,7 +69,7 @@ struct ScoreSmem {
 
 static_assert(ScoreSmem<128>::kAlloc <= 232448, "scoring smem over budget");
 
-template <int D>
+template <int D, bool FUSED = false>
 __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __grid_constant__ ScoreParams P) {
     using SM = ScoreSmem<D>;
     constexpr int QS = SM::QS, NB = SM::NB;
@@ -63,6 +78,18 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
+    if (FUSED && static_cast<int>(blockIdx.x) >= P.n_score_ctas) {
+        // anchor rows into the packed buffer
+        const Layer &L = P.L;
+        const int b = blockIdx.x - P.n_score_ctas;
+        const int per_g = (L.a + kAnchorRowsPerCta - 1) / kAnchorRowsPerCta;
+        const int g = b / per_g, r0 = (b % per_g) * kAnchorRowsPerCta;
+        const int r1 = min(L.a, r0 + kAnchorRowsPerCta);
+        const int sh = region_shift(L, 0);
+        copy_rows<D>(L, P.K, P.V, P.PK, P.PV, g, r0, r1, threadIdx.x >> 5, blockDim.x >> 5,
+                     [&](int r) { return r - sh; });
+        return;
+    }
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::kOffBar);
     uint64_t *a_full = bars;
     uint64_t *q_full = a_full + 1;
@@ -185,7 +212,18 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_free[sb]);
-            if (n_rows == 32) {
+            if (n_rows == 32 && ((reinterpret_cast<uintptr_t>(lse2) & 15) == 0)) {
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 l4 = __ldg(reinterpret_cast<const float4 *>(lse2 + c));
+                    const float2 a0 = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v,
+                                            make_float2(-l4.x, -l4.y));
+                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(a0.x), ex2(a0.y)));
+                    const float2 a1 = ffma2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), sl2v,
+                                            make_float2(-l4.z, -l4.w));
+                    acc[((c >> 1) + 1) & 3] = fadd2(acc[((c >> 1) + 1) & 3], make_float2(ex2(a1.x), ex2(a1.y)));
+                }
+            } else if (n_rows == 32) {
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const float2 nl = make_float2(-__ldg(lse2 + c), -__ldg(lse2 + c + 1));
@@ -219,6 +257,48 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+    if constexpr (FUSED) {
+        // The last CTA of (chunk u, KV head g) to finish selects and gathers.
+        __shared__ int s_last;
+        __threadfence();  // this CTA's scores, before its count
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const int n_tiles = P.tile_begin[u + 1] - P.tile_begin[u];
+            s_last = atomicAdd(&P.counters[u * L.Hkv + g], 1) == n_tiles - 1;
+        }
+        __syncthreads();
+        if (s_last) {
+            __threadfence();  // every other CTA's scores of (u, g), after their counts
+            // The tiles' shared memory is free: the rank keys go there.
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            const int l_eff = select_chunk(L, P.scores, P.idx, u, g, reinterpret_cast<uint32_t *>(smem),
+                                           SM::kOffBar / 4);
+            __syncthreads();
+            const int32_t *sel = P.idx + (static_cast<size_t>(u) * L.Hkv + g) * L.l;
+            const int p0 = L.pcum[u], sh = region_shift(L, 1 + u);
+            copy_rows<D>(L, P.K, P.V, P.PK, P.PV, g, p0, p0 + l_eff, warp, blockDim.x >> 5,
+                         [&](int r) { return sel[r - p0] - sh; });
+            if (threadIdx.x == 0) P.counters[u * L.Hkv + g] = 0;  // ready for the next launch
+        }
+    }
+}
+
+// Row-normalised scores: the base-2 log-sum-exp of every query row over all the
+// segments it attends, seg[s][h][i] combined over s (anchor s = 0 only if
+// a > 0, chunks s = 1..2H, query block s = 2H+1), written for every producing
+// chunk u so that the scoring pass reads it like a per-chunk statistic.
+__global__ void row_lse_kernel(const Layer L, const float *seg, float *stats) {
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;  // h * q + i
+    const int rows = L.Hq * L.q;
+    if (r >= rows) return;
+    const int s0 = L.a > 0 ? 0 : 1, s1 = L.n_chunks + 1;
+    float m = -INFINITY;
+    for (int s = s0; s <= s1; ++s) m = fmaxf(m, seg[static_cast<size_t>(s) * rows + r]);
+    float sum = 0.f;
+    if (m != -INFINITY)
+        for (int s = s0; s <= s1; ++s) sum += exp2f(seg[static_cast<size_t>(s) * rows + r] - m);
+    const float lse = (m == -INFINITY) ? -INFINITY : m + log2f(sum);
+    for (int u = 0; u < L.n_chunks - 1; ++u) stats[static_cast<size_t>(u) * rows + r] = lse;
 }
 
 }  // namespace spava

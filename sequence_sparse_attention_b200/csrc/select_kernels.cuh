@@ -59,19 +59,23 @@ constexpr int kSelectThreads = 1024;
 // The value a key is ranked by: its score, or with pooling (L.pool = w >= 3)
 // the sum of the scores of the w keys centred on it inside the chunk, added in
 // ascending order with plain fp32 adds (the window mean with zero padding up to
-// the factor 1/w, which does not change the ranking).
+// the factor 1/w, which does not change the ranking).  Scores are read through
+// L2 (another CTA of the same launch may have written them).
 __device__ __forceinline__ float rank_value(const float *S, int n, int j, int pool) {
-    if (pool <= 1) return S[j];
+    if (pool <= 1) return __ldcg(S + j);
     const int h = pool >> 1;
     const int k0 = j - h < 0 ? 0 : j - h, k1 = j + h < n ? j + h : n - 1;
     float s = 0.f;
-    for (int k = k0; k <= k1; ++k) s = __fadd_rn(s, S[k]);
+    for (int k = k0; k <= k1; ++k) s = __fadd_rn(s, __ldcg(S + k));
     return s;
 }
 
 // The selection of one (chunk u, KV head g) by the whole CTA; returns l_eff.
+// `keys` (shared memory, room for `cap` entries, or null): when the chunk
+// fits, each key's ordered rank value is computed once into it and the five
+// passes read it from there.
 __device__ __forceinline__ int select_chunk(const Layer &L, const float *scores, int32_t *idx, int u,
-                                            int g) {
+                                            int g, uint32_t *keys = nullptr, int cap = 0) {
     __shared__ int hist[256];
     __shared__ int warp_sums[32];
     __shared__ int s_digit, s_need, s_total;
@@ -88,6 +92,14 @@ __device__ __forceinline__ int select_chunk(const Layer &L, const float *scores,
         for (int r = tid; r < n; r += blockDim.x) out[r] = base + r;
         return l_eff;
     }
+    const bool cached = keys != nullptr && n <= cap;
+    if (cached) {
+        for (int j = tid; j < n; j += blockDim.x) keys[j] = ordered_key(rank_value(S, n, j, L.pool));
+        __syncthreads();
+    }
+    auto key_of = [&](int j) -> uint32_t {
+        return cached ? keys[j] : ordered_key(rank_value(S, n, j, L.pool));
+    };
 
     uint32_t prefix = 0, mask = 0;
     int need = l_eff;
@@ -95,7 +107,7 @@ __device__ __forceinline__ int select_chunk(const Layer &L, const float *scores,
         if (tid < 256) hist[tid] = 0;
         __syncthreads();
         for (int j = tid; j < n; j += blockDim.x) {
-            const uint32_t k = ordered_key(rank_value(S, n, j, L.pool));
+            const uint32_t k = key_of(j);
             if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
         }
         __syncthreads();
@@ -124,7 +136,7 @@ __device__ __forceinline__ int select_chunk(const Layer &L, const float *scores,
     const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
     int gt = 0, eq = 0;
     for (int j = j0; j < j1; ++j) {
-        const uint32_t k = ordered_key(rank_value(S, n, j, L.pool));
+        const uint32_t k = key_of(j);
         gt += k > T;
         eq += k == T;
     }
@@ -133,7 +145,7 @@ __device__ __forceinline__ int select_chunk(const Layer &L, const float *scores,
     int pos = block_exclusive_scan(gt + take_eq, warp_sums, &s_total);
     int taken = 0;
     for (int j = j0; j < j1; ++j) {
-        const uint32_t k = ordered_key(rank_value(S, n, j, L.pool));
+        const uint32_t k = key_of(j);
         if (k > T || (k == T && taken < take_eq)) {
             out[pos++] = base + j;
             taken += (k == T);
@@ -150,10 +162,13 @@ __device__ __forceinline__ int nth_owned_producer(const Layer &L, int k) {
     return -1;
 }
 
+// Dynamic shared memory of the selection kernels: room for the rank keys of
+// the longest chunk (0 if it does not fit; the passes then recompute them).
 __global__ void __launch_bounds__(kSelectThreads) topk_kernel(const Layer L, const float *scores,
-                                                              int32_t *idx) {
+                                                              int32_t *idx, int key_cap) {
+    extern __shared__ uint32_t sel_keys[];
     const int u = nth_owned_producer(L, blockIdx.x / L.Hkv);
-    if (u >= 0) select_chunk(L, scores, idx, u, blockIdx.x % L.Hkv);
+    if (u >= 0) select_chunk(L, scores, idx, u, blockIdx.x % L.Hkv, sel_keys, key_cap);
 }
 
 // Copies packed rows [r0, r1) of KV head g from the local token rows src(r): one warp
@@ -195,13 +210,14 @@ constexpr int kAnchorRowsPerCta = 256;
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) select_pack_kernel(
     const Layer L, const float *scores, int32_t *idx, const __nv_bfloat16 *K,
-    const __nv_bfloat16 *V, __nv_bfloat16 *PK, __nv_bfloat16 *PV, int n_sel_ctas) {
+    const __nv_bfloat16 *V, __nv_bfloat16 *PK, __nv_bfloat16 *PV, int n_sel_ctas, int key_cap) {
+    extern __shared__ uint32_t sel_keys[];
     const int n_sel = n_sel_ctas;
     const int warp = threadIdx.x >> 5, n_warps = blockDim.x >> 5;
     if (static_cast<int>(blockIdx.x) < n_sel) {
         const int u = nth_owned_producer(L, blockIdx.x / L.Hkv), g = blockIdx.x % L.Hkv;
         if (u < 0) return;
-        const int l_eff = select_chunk(L, scores, idx, u, g);
+        const int l_eff = select_chunk(L, scores, idx, u, g, sel_keys, key_cap);
         __syncthreads();
         const int32_t *sel = idx + (static_cast<size_t>(u) * L.Hkv + g) * L.l;
         const int p0 = L.pcum[u], sh = region_shift(L, 1 + u);

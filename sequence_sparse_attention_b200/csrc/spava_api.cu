@@ -12,7 +12,6 @@
 
 #include "../../include/spava.h"
 #include "attn_kernel.cuh"
-#include "stats_kernel.cuh"
 #include "plan.cuh"
 #include "score_kernel.cuh"
 #include "select_kernels.cuh"
@@ -150,25 +149,24 @@ int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int r
             if (seg_held(s)) push(kQueryPart, s, n_qrt);
     }
     std::stable_sort(gs.begin(), gs.end(), [](const G &x, const G &y) { return x.cost > y.cost; });
-    // The statistics pass runs one row tile per CTA, the attention two.
+    // Work items of two 128-row tiles each (statistics pass and attention alike).
     int begin = 0, n = 0;
     for (auto &g : gs) {
         g.g.item_begin = begin;
-        begin += stats ? g.g.n_rt * L.Hq : pair_items(g.g.n_rt, L.G) * L.Hkv;
+        begin += pair_items(g.g.n_rt, L.G) * L.Hkv;
         out[n++] = g.g;
     }
     return n;
 }
 
-int64_t plan_items(const Group *g, int n, const Layer &L, bool stats) {
+int64_t plan_items(const Group *g, int n, const Layer &L, bool /*stats*/) {
     if (!n) return 0;
-    const int per = stats ? g[n - 1].n_rt * L.Hq : pair_items(g[n - 1].n_rt, L.G) * L.Hkv;
-    return static_cast<int64_t>(g[n - 1].item_begin) + per;
+    return static_cast<int64_t>(g[n - 1].item_begin) + pair_items(g[n - 1].n_rt, L.G) * L.Hkv;
 }
 
 // ---------------------------------------------------------------- workspace
 struct WsLayout {
-    size_t status, stats, scores, idx, pk, pv, part_o, part_lse, total;
+    size_t status, stats, scores, idx, pk, pv, part_o, part_lse, counters, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -185,6 +183,7 @@ WsLayout ws_layout(const Layer &L) {
     w.pv = take(2 * size_t(L.Hkv) * L.L * L.d);
     w.part_o = take(sizeof(float) * size_t(L.n_chunks + 2) * L.Hq * L.q * L.d);
     w.part_lse = take(sizeof(float) * size_t(L.n_chunks + 2) * L.Hq * L.q);
+    w.counters = take(sizeof(int32_t) * size_t(L.n_chunks - 1) * L.Hkv);
     w.total = o;
     return w;
 }
@@ -269,31 +268,25 @@ spava_status launched() {
 // ---------------------------------------------------------------- launches
 template <int D, bool STATS>
 spava_status launch_attn(AttnParams &p, cudaStream_t st) {
-    const int64_t items = plan_items(p.groups, p.n_groups, p.L, STATS);
+    const int64_t items = plan_items(p.groups, p.n_groups, p.L, false);
     if (items == 0) return SPAVA_OK;
     if (items >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
-    if (STATS) {
-        using SM = StatsSmem<D>;
-        SPAVA_TRY(set_smem(stats_kernel<D>, SM::kAlloc));
-        stats_kernel<D><<<static_cast<unsigned>(items), kStatsThreads, SM::kAlloc, st>>>(p);
-    } else {
-        using SM = AttnSmem<D>;
-        // Persistent grid: one CTA per SM (the shared memory allows no more),
-        // each claiming items from the queue in the workspace.
-        int dev = 0, n_sm = 148;
-        SPAVA_CUDA(cudaGetDevice(&dev));
-        SPAVA_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
-        p.n_items = static_cast<int32_t>(items);
-        SPAVA_CUDA(cudaMemsetAsync(p.queue, 0, sizeof(int), st));
-        // The kernel's register split draws on the pool its launch allocates;
-        // refuse to launch a build whose per-thread count would leave it short.
-        cudaFuncAttributes fa;
-        SPAVA_CUDA(cudaFuncGetAttributes(&fa, attn_kernel<D>));
-        if (fa.numRegs < kLaunchRegs) return SPAVA_ERR_UNSUPPORTED;
-        SPAVA_TRY(set_smem(attn_kernel<D>, SM::kAlloc));
-        const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, n_sm));
-        attn_kernel<D><<<grid, kAttnThreads, SM::kAlloc, st>>>(p);
-    }
+    using SM = AttnSmem<D>;
+    // Persistent grid: one CTA per SM (the shared memory allows no more), each
+    // claiming items from the queue counter p.queue.
+    int dev = 0, n_sm = 148;
+    SPAVA_CUDA(cudaGetDevice(&dev));
+    SPAVA_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+    p.n_items = static_cast<int32_t>(items);
+    SPAVA_CUDA(cudaMemsetAsync(p.queue, 0, sizeof(int), st));
+    // The kernel's register split draws on the pool its launch allocates;
+    // refuse to launch a build whose per-thread count would leave it short.
+    cudaFuncAttributes fa;
+    SPAVA_CUDA(cudaFuncGetAttributes(&fa, attn_kernel<D, STATS>));
+    if (fa.numRegs < kLaunchRegs) return SPAVA_ERR_UNSUPPORTED;
+    SPAVA_TRY(set_smem(attn_kernel<D, STATS>, SM::kAlloc));
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(items, n_sm));
+    attn_kernel<D, STATS><<<grid, kAttnThreads, SM::kAlloc, st>>>(p);
     return launched();
 }
 
@@ -313,39 +306,11 @@ spava_status run_stats(const Layer &L, const void *q, const void *k, char *ws, c
     float *stats = reinterpret_cast<float *>(ws + w.stats);
     p.stats = L.norm ? reinterpret_cast<float *>(ws + w.part_lse) : stats;
     p.status = reinterpret_cast<int *>(ws + w.status);
+    p.queue = reinterpret_cast<int *>(ws + w.status + 128);
     SPAVA_TRY(L.d == 128 ? launch_attn<128, true>(p, st) : launch_attn<64, true>(p, st));
     if (!L.norm) return SPAVA_OK;
     const int rows = L.Hq * L.q;
     row_lse_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, st>>>(L, p.stats, stats);
-    return launched();
-}
-
-spava_status run_scores(const Layer &L, const void *q, const void *k, float *scores, char *ws,
-                        cudaStream_t st) {
-    const WsLayout w = ws_layout(L);
-    ScoreParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.L = L;
-    SPAVA_TRY(map_tokens(&p.tmQ, q, L, L.Hq));
-    SPAVA_TRY(map_tokens(&p.tmK, k, L, L.Hkv));
-    p.stats = reinterpret_cast<const float *>(ws + w.stats);
-    p.scores = scores;
-    p.status = reinterpret_cast<int *>(ws + w.status);
-    int tiles = 0;
-    for (int u = 0; u < L.n_chunks - 1; ++u) {
-        p.tile_begin[u] = tiles;
-        if (owns(L, u)) tiles += cdiv(L.off[u + 1] - L.off[u], 128);
-    }
-    p.tile_begin[L.n_chunks - 1] = tiles;
-    const int64_t blocks = static_cast<int64_t>(tiles) * L.Hkv;
-    if (blocks == 0) return SPAVA_OK;
-    if (L.d == 128) {
-        SPAVA_TRY(set_smem(score_kernel<128>, ScoreSmem<128>::kAlloc));
-        score_kernel<128><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<128>::kAlloc, st>>>(p);
-    } else {
-        SPAVA_TRY(set_smem(score_kernel<64>, ScoreSmem<64>::kAlloc));
-        score_kernel<64><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<64>::kAlloc, st>>>(p);
-    }
     return launched();
 }
 
@@ -356,10 +321,70 @@ int owned_producers(const Layer &L) {
     return n;
 }
 
+// Shared memory for the rank keys of the longest producing chunk held here
+// (0 if it does not fit: the selection passes then recompute them).
+int select_key_cap(const Layer &L) {
+    int n = 0;
+    for (int u = 0; u < L.n_chunks - 1; ++u)
+        if (owns(L, u)) n = std::max(n, L.off[u + 1] - L.off[u]);
+    return n * 4 <= kMaxDynSmem - 4096 ? n : 0;
+}
+
+// Query-to-context scores of the producing chunks held here, normalised by
+// `stats` ([2H-1, Hq, q] base-2 log-sum-exps).  fused: the same launch also
+// selects every (chunk, KV head)'s passing block into idx and gathers it,
+// and the anchor rows, into the packed buffers pk / pv.
+spava_status run_scores(const Layer &L, const void *q, const void *k, const float *stats, float *scores,
+                        char *ws, cudaStream_t st, bool fused = false, int32_t *idx = nullptr,
+                        const void *v = nullptr, void *pk = nullptr, void *pv = nullptr) {
+    const WsLayout w = ws_layout(L);
+    ScoreParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.L = L;
+    SPAVA_TRY(map_tokens(&p.tmQ, q, L, L.Hq));
+    SPAVA_TRY(map_tokens(&p.tmK, k, L, L.Hkv));
+    p.stats = stats;
+    p.scores = scores;
+    p.status = reinterpret_cast<int *>(ws + w.status);
+    int tiles = 0;
+    for (int u = 0; u < L.n_chunks - 1; ++u) {
+        p.tile_begin[u] = tiles;
+        if (owns(L, u)) tiles += cdiv(L.off[u + 1] - L.off[u], 128);
+    }
+    p.tile_begin[L.n_chunks - 1] = tiles;
+    const int64_t score_ctas = static_cast<int64_t>(tiles) * L.Hkv;
+    int64_t blocks = score_ctas;
+    if (fused) {
+        p.counters = reinterpret_cast<int *>(ws + w.counters);
+        p.idx = idx;
+        p.K = static_cast<const __nv_bfloat16 *>(k);
+        p.V = static_cast<const __nv_bfloat16 *>(v);
+        p.PK = static_cast<__nv_bfloat16 *>(pk);
+        p.PV = static_cast<__nv_bfloat16 *>(pv);
+        p.n_score_ctas = static_cast<int32_t>(score_ctas);
+        blocks += L.a > 0 ? static_cast<int64_t>(L.Hkv) * cdiv(L.a, kAnchorRowsPerCta) : 0;
+        SPAVA_CUDA(cudaMemsetAsync(p.counters, 0, sizeof(int32_t) * size_t(L.n_chunks - 1) * L.Hkv, st));
+    }
+    if (blocks == 0) return SPAVA_OK;
+    if (blocks >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
+    auto go = [&](auto kernel, int smem) -> spava_status {
+        SPAVA_TRY(set_smem(kernel, smem));
+        kernel<<<static_cast<unsigned>(blocks), kScoreBlockThreads, smem, st>>>(p);
+        return launched();
+    };
+    if (L.d == 128)
+        return fused ? go(score_kernel<128, true>, ScoreSmem<128>::kAlloc)
+                     : go(score_kernel<128, false>, ScoreSmem<128>::kAlloc);
+    return fused ? go(score_kernel<64, true>, ScoreSmem<64>::kAlloc)
+                 : go(score_kernel<64, false>, ScoreSmem<64>::kAlloc);
+}
+
 spava_status run_topk(const Layer &L, const float *scores, int32_t *idx, cudaStream_t st) {
     const int blocks = owned_producers(L) * L.Hkv;
     if (blocks == 0 || L.l == 0) return SPAVA_OK;
-    topk_kernel<<<blocks, kSelectThreads, 0, st>>>(L, scores, idx);  // pools on the fly (L.pool)
+    const int cap = select_key_cap(L);
+    SPAVA_TRY(set_smem(topk_kernel, cap * 4));
+    topk_kernel<<<blocks, kSelectThreads, cap * 4, st>>>(L, scores, idx, cap);  // pools on the fly (L.pool)
     return launched();
 }
 
@@ -397,12 +422,16 @@ spava_status run_select_pack(const Layer &L, const float *scores, int32_t *idx, 
     auto V = static_cast<const __nv_bfloat16 *>(v);
     auto PK = static_cast<__nv_bfloat16 *>(pk);
     auto PV = static_cast<__nv_bfloat16 *>(pv);
-    if (L.d == 128)
-        select_pack_kernel<128><<<blocks, kSelectThreads, 0, st>>>(L, scores, idx, K, V, PK, PV,
-                                                                   static_cast<int>(n_sel));
-    else
-        select_pack_kernel<64><<<blocks, kSelectThreads, 0, st>>>(L, scores, idx, K, V, PK, PV,
-                                                                  static_cast<int>(n_sel));
+    const int cap = select_key_cap(L);
+    if (L.d == 128) {
+        SPAVA_TRY(set_smem(select_pack_kernel<128>, cap * 4));
+        select_pack_kernel<128><<<blocks, kSelectThreads, cap * 4, st>>>(L, scores, idx, K, V, PK, PV,
+                                                                         static_cast<int>(n_sel), cap);
+    } else {
+        SPAVA_TRY(set_smem(select_pack_kernel<64>, cap * 4));
+        select_pack_kernel<64><<<blocks, kSelectThreads, cap * 4, st>>>(L, scores, idx, K, V, PK, PV,
+                                                                        static_cast<int>(n_sel), cap);
+    }
     return launched();
 }
 
@@ -447,22 +476,57 @@ spava_status run_attn(const Layer &L, const void *q, const void *k, const void *
     return run_merge(L, o, lse, ws, st);
 }
 
-// Scoring, selection and gather: everything of the layer before the attention.
-// Scoring reads only K and the query block's Q rows; if `v_ready` is given, the
-// gather (the first step that reads V) waits for it.
+// Scoring, selection and gather: everything of the layer before the attention,
+// from the statistics pass.  Scoring reads only K and the query block's Q rows;
+// with `v_ready` (the host entry point's copy pipeline) the selection and the
+// gather -- the first step that reads V -- run as their own launch after it,
+// otherwise in the scoring launch.
 spava_status run_front(const Layer &L, const void *q, const void *k, const void *v,
                        int32_t *idx_out, char *w, cudaStream_t st, cudaEvent_t v_ready = nullptr) {
     const WsLayout lay = ws_layout(L);
     float *scores = reinterpret_cast<float *>(w + lay.scores);
+    const float *stats = reinterpret_cast<const float *>(w + lay.stats);
     int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + lay.idx);
     if (L.n_chunks > 1 && L.l > 0) {
         SPAVA_TRY(run_stats(L, q, k, w, st));
-        SPAVA_TRY(run_scores(L, q, k, scores, w, st));
-        if (v_ready) SPAVA_CUDA(cudaStreamWaitEvent(st, v_ready, 0));
+        if (!v_ready)
+            return run_scores(L, q, k, stats, scores, w, st, true, idx, v, w + lay.pk, w + lay.pv);
+        SPAVA_TRY(run_scores(L, q, k, stats, scores, w, st));
+        SPAVA_CUDA(cudaStreamWaitEvent(st, v_ready, 0));
         return run_select_pack(L, scores, idx, k, v, w + lay.pk, w + lay.pv, st);
     }
     if (v_ready) SPAVA_CUDA(cudaStreamWaitEvent(st, v_ready, 0));
     return run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st);  // anchor rows only
+}
+
+// The whole layer on device buffers, in the order of the pages' fused forward
+// ("Forward Fuso di Contesto e Query"): first the work that needs no passing
+// block -- the anchor rows and the query rows' partials over every segment,
+// whose per-chunk log-sum-exps ARE the scoring's normaliser (the statistics
+// pass computes the same values bit for bit) -- then scoring fused with the
+// selection and the gather, then the context rows and the query-row merge.
+spava_status run_layer(const Layer &L, const void *q, const void *k, const void *v, void *o,
+                       float *lse, int32_t *idx_out, char *w, cudaStream_t st) {
+    const WsLayout lay = ws_layout(L);
+    if (!(L.n_chunks > 1 && L.l > 0)) {
+        SPAVA_TRY(run_front(L, q, k, v, idx_out, w, st));
+        return run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st);
+    }
+    SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st, 0, INT32_MAX,
+                       (1u << kAnchor) | (1u << kQueryPart), false));
+    float *part_lse = reinterpret_cast<float *>(w + lay.part_lse);
+    const float *stats = part_lse + size_t(L.Hq) * L.q;  // segment 1 + u = chunk u
+    if (L.norm) {  // each row's log-sum-exp over all its segments
+        float *row = reinterpret_cast<float *>(w + lay.stats);
+        const int rows = L.Hq * L.q;
+        row_lse_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, st>>>(L, part_lse, row);
+        SPAVA_TRY(launched());
+        stats = row;
+    }
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + lay.idx);
+    SPAVA_TRY(run_scores(L, q, k, stats, reinterpret_cast<float *>(w + lay.scores), w, st, true, idx, v,
+                         w + lay.pk, w + lay.pv));
+    return run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st, 0, INT32_MAX, 1u << kCtx, true);
 }
 
 // Row groups of the copy/compute pipeline of the host entry point, in the
@@ -531,8 +595,9 @@ spava_status spava_score(const spava_config *cfg, const void *q, const void *k, 
     SPAVA_TRY(check_ptr(scores));
     SPAVA_TRY(check_ws(L, ws, ws_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    SPAVA_TRY(run_stats(L, q, k, static_cast<char *>(ws), st));
-    return run_scores(L, q, k, scores, static_cast<char *>(ws), st);
+    char *w = static_cast<char *>(ws);
+    SPAVA_TRY(run_stats(L, q, k, w, st));
+    return run_scores(L, q, k, reinterpret_cast<const float *>(w + ws_layout(L).stats), scores, w, st);
 }
 
 spava_status spava_topk_select(const spava_config *cfg, const float *scores, int32_t *idx,
@@ -589,11 +654,7 @@ spava_status spava_prefill_attention(const spava_config *cfg, const void *q, con
     SPAVA_TRY(check_ptr(lse, false));
     SPAVA_TRY(check_ptr(idx_out, false));
     SPAVA_TRY(check_ws(L, ws, ws_bytes));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    char *w = static_cast<char *>(ws);
-    SPAVA_TRY(run_front(L, q, k, v, idx_out, w, st));
-    const WsLayout lay = ws_layout(L);
-    return run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st);
+    return run_layer(L, q, k, v, o, lse, idx_out, static_cast<char *>(ws), static_cast<cudaStream_t>(stream));
 }
 
 spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q_host,
@@ -1087,7 +1148,7 @@ spava_status spava_shard_merge(const spava_config *cfg, int32_t rank, int32_t wo
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
-constexpr size_t kNoAllocStatusBytes = 256;                // status word, then statistics
+constexpr size_t kNoAllocStatusBytes = 256;  // status word (byte 0), work-item counter (byte 128)
 
 static __device__ __align__(256) unsigned char g_score_scratch[kNoAllocScratchBytes];
 
@@ -1134,6 +1195,7 @@ extern "C" spava_status spava_score_noalloc(const spava_config *cfg, const void 
     sp.n_groups = plan_attention(L, true, sp.groups);
     sp.stats = stats;
     sp.status = status;
+    sp.queue = reinterpret_cast<int *>(base + 128);  // work-item counter, inside the status block
     SPAVA_TRY(L.d == 128 ? launch_attn<128, true>(sp, st) : launch_attn<64, true>(sp, st));
 
     ScoreParams p;
