@@ -255,9 +255,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     if (warp == kProducerWarp && lane == 0) {
         tma_prefetch(&P.tmQ);
         tma_prefetch(&P.tmK);
-        tma_prefetch(&P.tmV);
-        tma_prefetch(&P.tmPK);
-        tma_prefetch(&P.tmPV);
+        if (!STATS) {  // the statistics pass encodes only the Q and K maps
+            tma_prefetch(&P.tmV);
+            tma_prefetch(&P.tmPK);
+            tma_prefetch(&P.tmPV);
+        }
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -578,8 +580,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
 
         // ------------------------------------------------------------ epilogue
         if (STATS) {
-            // The row's base-2 log-sum-exp over the item's keys.
-            if (ok && t < row_end) {
+            // The row's base-2 log-sum-exp over the item's keys (tile B may be
+            // absent: TB = 0, no head).
+            if (ok && TX > 0 && t < row_end) {
                 const int i = t - (L.N - L.q);
                 P.stats[(static_cast<size_t>(it.sub) * L.Hq + hx) * L.q + i] =
                     (l_run > 0.f) ? __fadd_rn(m_run, __log2f(l_run)) : -INFINITY;
