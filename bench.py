@@ -42,9 +42,12 @@ from sequence_sparse_attention_b200.synth import WORKLOADS, chunk_offsets, make_
 
 METRIC = "approx-attn prefill tokens/s per layer on 1 B200; % BF16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# Kernels one spava_prefill_attention call launches: statistics, scores, the
-# fused top-l + gather, attention, query merge.
-KERNELS_PER_STEP = 5
+# Kernels one spava_prefill_attention call launches: the anchor rows and
+# query partials (attention kernel), scoring fused with top-l and gather, the
+# context rows (attention kernel), the query merge.
+KERNELS_PER_STEP = 4
+# The four separate steps: statistics + scores, top-l, gather, attention + merge.
+KERNELS_PER_SPLIT_STEP = 6
 
 # DRAM traffic of one attention launch on the 128K layer (dram__bytes_read.sum
 # + dram__bytes_write.sum of a single-pass ncu capture); valid only while the
@@ -454,7 +457,7 @@ def run_ours(args, world, rank, local):
         "tensor_peak_frac": {"of_burst": achieved / peak, "of_sustained": achieved / sustained,
                              "of_nominal_2250": achieved / 2250.0},
         "e2e": e2e, "gpu_launches": KERNELS_PER_STEP * args.steps,
-        "gpu_launches_split_region": 6 * args.steps, "clocks": clocks,
+        "gpu_launches_split_region": KERNELS_PER_SPLIT_STEP * args.steps, "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, cores, _ = oracle_sample(w, args.cpu_budget, oracle_inputs(w, Q, K, V))
