@@ -10,11 +10,21 @@
 // the query-row partial of chunk u ("Forward Fuso di Contesto e Query").
 // Equivalently: softmax over the chunk, summed over query rows and group heads.
 //
-// One CTA = 128 keys of one chunk and one KV head.  The product is formed
-// transposed, S^T = K Q^T (M = 128 keys, N = 128 query rows of one head per
-// block, K = d), so that TMEM lane j holds key j and each thread sums its own
-// key's probabilities without any cross-thread reduction; the summation order
-// is fixed, so the result is deterministic.
+// One CTA = a score unit: two 128-key tiles (the last unit of a chunk may have
+// one) of one chunk and one KV head.  The product is formed transposed,
+// S^T = K Q^T (M = 128 keys, N = 128 query rows of one head per block, K = d),
+// so that TMEM lane j holds key j and each thread sums its own keys'
+// probabilities without any cross-thread reduction; both tiles of a unit take
+// the same query block from shared memory and the same log-sum-exp loads.  The
+// summation order is fixed, so the result is deterministic.
+//
+// The exponentials are MUFU-bound (one per 2*d tensor FLOPs, against a MUFU
+// rate of 16 per SM per clock), with the FMA pipe idle: a quarter of them run
+// on the FMA pipe instead, as 2^a = 2^n * p(f) with n = round(a), f = a - n in
+// [-1/2, 1/2] (Cody-Waite style reduction; n is read off the low mantissa bits
+// of a + 1.5*2^23) and p a degree-4 polynomial fitted to 2^f in relative error
+// by Lawson's iteratively reweighted least squares (fit_exp2_poly.py in this
+// directory; max relative error 2.7e-6 in fp32 Horner form).
 //
 // FUSED = true also selects and gathers (the layer entry points): the CTA that
 // writes the last 128-key tile of a (chunk, KV head) -- counted with an atomic
@@ -36,43 +46,68 @@ struct ScoreParams {
     const float *stats;  // [2H-1, Hq, q] log2 domain
     float *scores;       // [Hkv, C]
     int *status;
-    int32_t tile_begin[kMaxChunks + 1];  // prefix of 128-key tiles over chunks u < 2H-1
+    int32_t unit_begin[kMaxChunks + 1];  // prefix of score units over chunks u < 2H-1
     // FUSED only
-    int *counters;       // [2H-1, Hkv] finished tiles, zero at launch
+    int *counters;       // [2H-1, Hkv] finished units, zero at launch
     int32_t *idx;        // [2H-1, Hkv, l]
     const __nv_bfloat16 *K, *V;
     __nv_bfloat16 *PK, *PV;  // [Hkv, L, D]
     int32_t n_score_ctas;
 };
 
+constexpr int kScoreTiles = 2;                  // 128-key tiles per score unit
 constexpr int kScoreWarps = 16;                 // 4 per TMEM lane quarter
 constexpr int kScoreThreads = kScoreWarps * 32;
 constexpr int kScoreProducer = kScoreWarps;
 constexpr int kScoreMma = kScoreWarps + 1;
 constexpr int kScoreBlockThreads = (kScoreWarps + 2) * 32;
+constexpr int kPolyEvery = 4;                   // every 4th exponential pair on the FMA pipe
+
+// Coefficients of p(f) ~ 2^f on [-1/2, 1/2] (fit_exp2_poly.py).
+constexpr float kExp2C0 = 0.9999992847442627f;
+constexpr float kExp2C1 = 0.6931217908859253f;
+constexpr float kExp2C2 = 0.240247443318367f;
+constexpr float kExp2C3 = 0.05591782182455063f;
+constexpr float kExp2C4 = 0.009570080786943436f;
+
+// 2^a for a pair of arguments on the FMA pipe.  Arguments below -126 are taken
+// as -126 (2^-126 and below contribute nothing to a score).
+__device__ __forceinline__ float2 exp2_fma2(float2 a) {
+    a = make_float2(fmaxf(a.x, -126.f), fmaxf(a.y, -126.f));
+    const float2 shifter = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
+    const float2 t = fadd2(a, shifter);                            // n in the low mantissa bits
+    const float2 n = fadd2(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = ffma2(n, make_float2(-1.f, -1.f), a);        // a - n, exact
+    float2 p = ffma2(make_float2(kExp2C4, kExp2C4), f, make_float2(kExp2C3, kExp2C3));
+    p = ffma2(p, f, make_float2(kExp2C2, kExp2C2));
+    p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
+    p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
+    // times 2^n: n added to the exponent field (t's low bits shifted into place)
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
 
 template <int D>
 struct ScoreSmem {
     static constexpr int kPanels = D / 64;
     static constexpr int kTile = 128 * D * 2;
     static constexpr int QS = 4;
-    static constexpr int NB = 4;  // TMEM S buffers
-    static constexpr int kOffK = 0;
-    static constexpr int kOffQ = kTile;
+    static constexpr int kOffK = 0;                        // the unit's key tiles
+    static constexpr int kOffQ = kScoreTiles * kTile;      // query-block ring
     static constexpr int kOffBar = kOffQ + QS * kTile;
-    static constexpr int kNumBar = 1 + 2 * QS + 2 * NB + 1;
-    static constexpr int kOffRed = kOffBar + kNumBar * 8;   // [4 parts][128 keys] partial sums
-    static constexpr int kOffMisc = kOffRed + 4 * 128 * 4;
+    static constexpr int kNumBar = 1 + 2 * QS + 2 * 2 + 1;
+    static constexpr int kOffRed = kOffBar + kNumBar * 8;  // [4 parts][256 keys] partial sums
+    static constexpr int kOffMisc = kOffRed + 4 * kScoreTiles * 128 * 4;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
 };
 
-static_assert(ScoreSmem<128>::kAlloc <= 232448, "scoring smem over budget");
+static_assert(ScoreSmem<128>::kAlloc + 2048 <= 232448, "scoring smem over budget");
 
 template <int D, bool FUSED = false>
 __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __grid_constant__ ScoreParams P) {
     using SM = ScoreSmem<D>;
-    constexpr int QS = SM::QS, NB = SM::NB;
+    constexpr int QS = SM::QS;
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, 128, 0, 0);
 
     extern __shared__ uint8_t smem_raw[];
@@ -94,22 +129,22 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
     uint64_t *a_full = bars;
     uint64_t *q_full = a_full + 1;
     uint64_t *q_empty = q_full + QS;
-    uint64_t *s_full = q_empty + QS;
-    uint64_t *s_free = s_full + NB;
-    uint64_t *mma_drain = s_free + NB;
+    uint64_t *s_full = q_empty + QS;  // [2]: S of both tiles of block b in buffer b & 1
+    uint64_t *s_free = s_full + 2;
+    uint64_t *mma_drain = s_free + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::kOffMisc + 4);
 
     const Layer &L = P.L;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // blockIdx.x = tile * Hkv + g, tiles enumerated over chunks u < 2H-1
+    // blockIdx.x = unit * Hkv + g, units enumerated over the chunks u < 2H-1
     const int g = blockIdx.x % L.Hkv;
-    const int tile = blockIdx.x / L.Hkv;
+    const int unit = blockIdx.x / L.Hkv;
     int u = 0;
-    while (u + 1 < L.n_chunks - 1 && tile >= P.tile_begin[u + 1]) ++u;
-    const int kt = tile - P.tile_begin[u];
-    const int key0 = L.off[u] + kt * 128;
-    const int n_valid = min(128, L.off[u + 1] - key0);
+    while (u + 1 < L.n_chunks - 1 && unit >= P.unit_begin[u + 1]) ++u;
+    const int key0 = L.off[u] + (unit - P.unit_begin[u]) * kScoreTiles * 128;
+    const int n_keys = min(kScoreTiles * 128, L.off[u + 1] - key0);  // 1 .. 256
+    const int nt = cdiv(n_keys, 128);                                // key tiles: 1 or 2
     const int n_rb = cdiv(L.q, 128);
     const int NBLK = L.G * n_rb;  // column blocks: (head in group, 128 query rows)
 
@@ -119,7 +154,7 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
             mbar_init(&q_full[i], 1);
             mbar_init(&q_empty[i], 1);
         }
-        for (int i = 0; i < NB; ++i) {
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&s_free[i], kScoreThreads);
         }
@@ -140,10 +175,12 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
 
     if (warp == kScoreProducer) {
         if (lane == 0) {
-            mbar_expect_tx(a_full, SM::kTile);
-            for (int p = 0; p < SM::kPanels; ++p)
-                tma_load_3d(smem + SM::kOffK + p * 16384, &P.tmK, p * 64, g, key0 - region_shift(L, 1 + u),
-                            a_full);
+            mbar_expect_tx(a_full, nt * SM::kTile);
+            const int krow = key0 - region_shift(L, 1 + u);  // local row of the unit's first key
+            for (int t = 0; t < nt; ++t)
+                for (int p = 0; p < SM::kPanels; ++p)
+                    tma_load_3d(smem + SM::kOffK + t * SM::kTile + p * 16384, &P.tmK, p * 64, g,
+                                krow + t * 128, a_full);
             int q_last[QS];
             for (int i = 0; i < QS; ++i) q_last[i] = -1;
             for (int b = 0; b < NBLK; ++b) {
@@ -163,92 +200,113 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
         }
     } else if (warp == kScoreMma) {
         if (lane == 0) {
-            const uint32_t a_base = smem_u32(smem + SM::kOffK);
+            const uint32_t k_base = smem_u32(smem + SM::kOffK);
             const uint32_t q_base = smem_u32(smem + SM::kOffQ);
             bool ok = mbar_wait(a_full, 0, ab);
             tc_fence_after();
             for (int b = 0; ok && b < NBLK; ++b) {
-                const int qs = b % QS, sb = b % NB;
+                const int qs = b % QS, pb = b & 1;
                 if (!mbar_wait(&q_full[qs], (b / QS) & 1, ab)) break;
-                if (b >= NB && !mbar_wait(&s_free[sb], ((b / NB) - 1) & 1, ab)) break;
+                if (b >= 2 && !mbar_wait(&s_free[pb], ((b >> 1) - 1) & 1, ab)) break;
                 tc_fence_after();
                 const uint32_t qb = q_base + qs * SM::kTile;
+                for (int t = 0; t < nt; ++t) {
+                    const uint32_t kb = k_base + t * SM::kTile;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + sb * 128, sdesc_sw128(a_base + off, 16, 1024),
-                           sdesc_sw128(qb + off, 16, 1024), kIdesc, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        mma_ss(tmem + pb * 256 + t * 128, sdesc_sw128(kb + off, 16, 1024),
+                               sdesc_sw128(qb + off, 16, 1024), kIdesc, kk > 0);
+                    }
                 }
                 tc_commit(&q_empty[qs]);
-                tc_commit(&s_full[sb]);
+                tc_commit(&s_full[pb]);
             }
             tc_commit(mma_drain);
             mbar_wait_drain(mma_drain, 0);
         }
         __syncwarp();
     } else {
-        // Warp w: keys 32*(w%4) .. +31 (its TMEM lane quarter), query-row columns
-        // 32*(w/4) .. +31 of every 128-column block; the four column parts of a
-        // key are added at the end.
+        // Warp w: keys 32*(w%4) .. +31 of each tile (its TMEM lane quarter),
+        // query-row columns 32*(w/4) .. +31 of every 128-column block; the four
+        // column parts of a key are added at the end.
         const int quarter = warp & 3, part = warp >> 2;
-        const int j = quarter * 32 + lane;  // key within the tile == TMEM lane
+        const int j = quarter * 32 + lane;  // key within a tile == TMEM lane
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const float2 sl2v = make_float2(L.scale_log2, L.scale_log2);
-        float2 acc[4];  // 8 independent partial sums, in packed pairs
+        float2 acc[kScoreTiles][4];  // per tile 8 independent partial sums, in packed pairs
 #pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
+        for (int t = 0; t < kScoreTiles; ++t)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[t][k] = make_float2(0.f, 0.f);
+        const bool two = nt > 1;  // CTA-uniform
+        // Exponentials of one pair of logits: pair k of the block (0..31 over
+        // both tiles) goes to the FMA pipe when k % kPolyEvery is the last slot.
+        auto add_pair = [&](int t, int c, float2 arg) {
+            const int k = t * 16 + (c >> 1);
+            const float2 p = (k % kPolyEvery == kPolyEvery - 1) ? exp2_fma2(arg)
+                                                                 : make_float2(ex2(arg.x), ex2(arg.y));
+            acc[t][(c >> 1) & 3] = fadd2(acc[t][(c >> 1) & 3], p);
+        };
         bool ok = true;
         for (int b = 0; b < NBLK; ++b) {
-            const int sb = b % NB;
+            const int pb = b & 1;
             const int h = g * L.G + b / n_rb;
             const int i0 = (b % n_rb) * 128 + part * 32;
             const float *lse2 = P.stats + (static_cast<size_t>(u) * L.Hq + h) * L.q + i0;
             const int n_rows = min(32, L.q - i0);  // may be <= 0 for the ragged last block
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (b / NB) & 1, ab));
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[pb], (b >> 1) & 1, ab));
             if (!ok) break;
             tc_fence_after();
-            uint32_t r[32];
-            tmem_ld32(lane_addr + sb * 128 + part * 32, r);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&s_free[sb]);
-            if (n_rows == 32 && ((reinterpret_cast<uintptr_t>(lse2) & 15) == 0)) {
+            // The two tiles' logits one after the other (32 registers each:
+            // 18 warps share each sub-partition's 16K registers).
+            const bool vec = n_rows == 32 && ((reinterpret_cast<uintptr_t>(lse2) & 15) == 0);
 #pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const float4 l4 = __ldg(reinterpret_cast<const float4 *>(lse2 + c));
-                    const float2 a0 = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v,
-                                            make_float2(-l4.x, -l4.y));
-                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(a0.x), ex2(a0.y)));
-                    const float2 a1 = ffma2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])), sl2v,
-                                            make_float2(-l4.z, -l4.w));
-                    acc[((c >> 1) + 1) & 3] = fadd2(acc[((c >> 1) + 1) & 3], make_float2(ex2(a1.x), ex2(a1.y)));
+            for (int t = 0; t < kScoreTiles; ++t) {
+                if (t > 0 && !two) break;
+                uint32_t r[32];
+                tmem_ld32(lane_addr + pb * 256 + t * 128 + part * 32, r);
+                tmem_wait_ld();
+                if (t + 1 == nt) {  // S buffer pb read completely
+                    tc_fence_before();
+                    mbar_arrive(&s_free[pb]);
                 }
-            } else if (n_rows == 32) {
+                if (vec) {
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float2 nl = make_float2(-__ldg(lse2 + c), -__ldg(lse2 + c + 1));
-                    const float2 arg = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v, nl);
-                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(arg.x), ex2(arg.y)));
-                }
-            } else {
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 l4 = __ldg(reinterpret_cast<const float4 *>(lse2 + c));
+                        add_pair(t, c, ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v,
+                                             make_float2(-l4.x, -l4.y)));
+                        add_pair(t, c + 2, ffma2(make_float2(__uint_as_float(r[c + 2]), __uint_as_float(r[c + 3])),
+                                                 sl2v, make_float2(-l4.z, -l4.w)));
+                    }
+                } else {
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float2 nl = make_float2(c < n_rows ? -__ldg(lse2 + c) : -INFINITY,
-                                                  c + 1 < n_rows ? -__ldg(lse2 + c + 1) : -INFINITY);
-                    const float2 arg = ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v, nl);
-                    acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(ex2(arg.x), ex2(arg.y)));
+                    for (int c = 0; c < 32; c += 2) {
+                        const float2 nl = make_float2(c < n_rows ? -__ldg(lse2 + c) : -INFINITY,
+                                                      c + 1 < n_rows ? -__ldg(lse2 + c + 1) : -INFINITY);
+                        add_pair(t, c, ffma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2v, nl));
+                    }
                 }
             }
         }
-        float *red = reinterpret_cast<float *>(smem + SM::kOffRed);
-        red[part * 128 + j] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-                              ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+        float *red = reinterpret_cast<float *>(smem + SM::kOffRed);  // [4 parts][256 keys]
+#pragma unroll
+        for (int t = 0; t < kScoreTiles; ++t)
+            red[part * 256 + t * 128 + j] = ((acc[t][0].x + acc[t][0].y) + (acc[t][1].x + acc[t][1].y)) +
+                                            ((acc[t][2].x + acc[t][2].y) + (acc[t][3].x + acc[t][3].y));
         // All score warps leave the loop together (the abort flag is CTA-wide and
         // every wait is bounded), so this barrier is always reached by all 512.
         bar_sync(1, kScoreThreads);
-        if (part == 0 && ok && j < n_valid)
-            P.scores[static_cast<size_t>(g) * L.C + (key0 - L.a) + j] =
-                (red[j] + red[128 + j]) + (red[256 + j] + red[384 + j]);
+        if (part == 0 && ok) {
+#pragma unroll
+            for (int t = 0; t < kScoreTiles; ++t) {
+                const int key = t * 128 + j;
+                if (key < n_keys)
+                    P.scores[static_cast<size_t>(g) * L.C + (key0 - L.a) + key] =
+                        (red[key] + red[256 + key]) + (red[512 + key] + red[768 + key]);
+            }
+        }
     }
 
     tc_fence_before();
@@ -263,8 +321,8 @@ __global__ void __launch_bounds__(kScoreBlockThreads, 1) score_kernel(const __gr
         __threadfence();  // this CTA's scores, before its count
         __syncthreads();
         if (threadIdx.x == 0) {
-            const int n_tiles = P.tile_begin[u + 1] - P.tile_begin[u];
-            s_last = atomicAdd(&P.counters[u * L.Hkv + g], 1) == n_tiles - 1;
+            const int n_units = P.unit_begin[u + 1] - P.unit_begin[u];
+            s_last = atomicAdd(&P.counters[u * L.Hkv + g], 1) == n_units - 1;
         }
         __syncthreads();
         if (s_last) {

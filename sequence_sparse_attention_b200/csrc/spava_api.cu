@@ -330,14 +330,22 @@ int select_key_cap(const Layer &L) {
     return n * 4 <= kMaxDynSmem - 4096 ? n : 0;
 }
 
+// What the fused scoring launch also needs: where the selection and the gather
+// go, and the finished-unit counters.
+struct FusedSelect {
+    int32_t *idx;
+    const void *v;
+    void *pk, *pv;
+    int *counters;
+};
+
 // Query-to-context scores of the producing chunks held here, normalised by
-// `stats` ([2H-1, Hq, q] base-2 log-sum-exps).  fused: the same launch also
-// selects every (chunk, KV head)'s passing block into idx and gathers it,
-// and the anchor rows, into the packed buffers pk / pv.
+// `stats` ([2H-1, Hq, q] base-2 log-sum-exps); `status`: the status word of the
+// bounded waits.  With `fused`, the same launch also selects every (chunk, KV
+// head)'s passing block into fused->idx and gathers it, and the anchor rows,
+// into the packed buffers.
 spava_status run_scores(const Layer &L, const void *q, const void *k, const float *stats, float *scores,
-                        char *ws, cudaStream_t st, bool fused = false, int32_t *idx = nullptr,
-                        const void *v = nullptr, void *pk = nullptr, void *pv = nullptr) {
-    const WsLayout w = ws_layout(L);
+                        int *status, cudaStream_t st, const FusedSelect *fused = nullptr) {
     ScoreParams p;
     std::memset(&p, 0, sizeof(p));
     p.L = L;
@@ -345,22 +353,22 @@ spava_status run_scores(const Layer &L, const void *q, const void *k, const floa
     SPAVA_TRY(map_tokens(&p.tmK, k, L, L.Hkv));
     p.stats = stats;
     p.scores = scores;
-    p.status = reinterpret_cast<int *>(ws + w.status);
-    int tiles = 0;
+    p.status = status;
+    int units = 0;  // score units: pairs of 128-key tiles of one chunk
     for (int u = 0; u < L.n_chunks - 1; ++u) {
-        p.tile_begin[u] = tiles;
-        if (owns(L, u)) tiles += cdiv(L.off[u + 1] - L.off[u], 128);
+        p.unit_begin[u] = units;
+        if (owns(L, u)) units += cdiv(cdiv(L.off[u + 1] - L.off[u], 128), kScoreTiles);
     }
-    p.tile_begin[L.n_chunks - 1] = tiles;
-    const int64_t score_ctas = static_cast<int64_t>(tiles) * L.Hkv;
+    p.unit_begin[L.n_chunks - 1] = units;
+    const int64_t score_ctas = static_cast<int64_t>(units) * L.Hkv;
     int64_t blocks = score_ctas;
     if (fused) {
-        p.counters = reinterpret_cast<int *>(ws + w.counters);
-        p.idx = idx;
+        p.counters = fused->counters;
+        p.idx = fused->idx;
         p.K = static_cast<const __nv_bfloat16 *>(k);
-        p.V = static_cast<const __nv_bfloat16 *>(v);
-        p.PK = static_cast<__nv_bfloat16 *>(pk);
-        p.PV = static_cast<__nv_bfloat16 *>(pv);
+        p.V = static_cast<const __nv_bfloat16 *>(fused->v);
+        p.PK = static_cast<__nv_bfloat16 *>(fused->pk);
+        p.PV = static_cast<__nv_bfloat16 *>(fused->pv);
         p.n_score_ctas = static_cast<int32_t>(score_ctas);
         blocks += L.a > 0 ? static_cast<int64_t>(L.Hkv) * cdiv(L.a, kAnchorRowsPerCta) : 0;
         SPAVA_CUDA(cudaMemsetAsync(p.counters, 0, sizeof(int32_t) * size_t(L.n_chunks - 1) * L.Hkv, st));
@@ -377,6 +385,17 @@ spava_status run_scores(const Layer &L, const void *q, const void *k, const floa
                      : go(score_kernel<128, false>, ScoreSmem<128>::kAlloc);
     return fused ? go(score_kernel<64, true>, ScoreSmem<64>::kAlloc)
                  : go(score_kernel<64, false>, ScoreSmem<64>::kAlloc);
+}
+
+// The same, with the workspace's status word and counters.
+spava_status run_scores_ws(const Layer &L, const void *q, const void *k, const float *stats, float *scores,
+                           char *ws, cudaStream_t st, bool fused = false, int32_t *idx = nullptr,
+                           const void *v = nullptr, void *pk = nullptr, void *pv = nullptr) {
+    const WsLayout w = ws_layout(L);
+    int *status = reinterpret_cast<int *>(ws + w.status);
+    if (!fused) return run_scores(L, q, k, stats, scores, status, st);
+    const FusedSelect f{idx, v, pk, pv, reinterpret_cast<int *>(ws + w.counters)};
+    return run_scores(L, q, k, stats, scores, status, st, &f);
 }
 
 spava_status run_topk(const Layer &L, const float *scores, int32_t *idx, cudaStream_t st) {
@@ -490,8 +509,8 @@ spava_status run_front(const Layer &L, const void *q, const void *k, const void 
     if (L.n_chunks > 1 && L.l > 0) {
         SPAVA_TRY(run_stats(L, q, k, w, st));
         if (!v_ready)
-            return run_scores(L, q, k, stats, scores, w, st, true, idx, v, w + lay.pk, w + lay.pv);
-        SPAVA_TRY(run_scores(L, q, k, stats, scores, w, st));
+            return run_scores_ws(L, q, k, stats, scores, w, st, true, idx, v, w + lay.pk, w + lay.pv);
+        SPAVA_TRY(run_scores_ws(L, q, k, stats, scores, w, st));
         SPAVA_CUDA(cudaStreamWaitEvent(st, v_ready, 0));
         return run_select_pack(L, scores, idx, k, v, w + lay.pk, w + lay.pv, st);
     }
@@ -524,8 +543,8 @@ spava_status run_layer(const Layer &L, const void *q, const void *k, const void 
         stats = row;
     }
     int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(w + lay.idx);
-    SPAVA_TRY(run_scores(L, q, k, stats, reinterpret_cast<float *>(w + lay.scores), w, st, true, idx, v,
-                         w + lay.pk, w + lay.pv));
+    SPAVA_TRY(run_scores_ws(L, q, k, stats, reinterpret_cast<float *>(w + lay.scores), w, st, true, idx, v,
+                            w + lay.pk, w + lay.pv));
     return run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, lse, w, st, 0, INT32_MAX, 1u << kCtx, true);
 }
 
@@ -597,7 +616,7 @@ spava_status spava_score(const spava_config *cfg, const void *q, const void *k, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *w = static_cast<char *>(ws);
     SPAVA_TRY(run_stats(L, q, k, w, st));
-    return run_scores(L, q, k, reinterpret_cast<const float *>(w + ws_layout(L).stats), scores, w, st);
+    return run_scores_ws(L, q, k, reinterpret_cast<const float *>(w + ws_layout(L).stats), scores, w, st);
 }
 
 spava_status spava_topk_select(const spava_config *cfg, const float *scores, int32_t *idx,
@@ -1198,30 +1217,7 @@ extern "C" spava_status spava_score_noalloc(const spava_config *cfg, const void 
     sp.queue = reinterpret_cast<int *>(base + 128);  // work-item counter, inside the status block
     SPAVA_TRY(L.d == 128 ? launch_attn<128, true>(sp, st) : launch_attn<64, true>(sp, st));
 
-    ScoreParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.L = L;
-    p.tmQ = sp.tmQ;
-    p.tmK = sp.tmK;
-    p.stats = stats;
-    p.scores = scores;
-    p.status = status;
-    int tiles = 0;
-    for (int u = 0; u < L.n_chunks - 1; ++u) {
-        p.tile_begin[u] = tiles;
-        tiles += cdiv(L.off[u + 1] - L.off[u], 128);
-    }
-    p.tile_begin[L.n_chunks - 1] = tiles;
-    const int64_t blocks = static_cast<int64_t>(tiles) * L.Hkv;
-    if (blocks == 0) return SPAVA_OK;
-    if (L.d == 128) {
-        SPAVA_TRY(set_smem(score_kernel<128>, ScoreSmem<128>::kAlloc));
-        score_kernel<128><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<128>::kAlloc, st>>>(p);
-    } else {
-        SPAVA_TRY(set_smem(score_kernel<64>, ScoreSmem<64>::kAlloc));
-        score_kernel<64><<<static_cast<unsigned>(blocks), kScoreBlockThreads, ScoreSmem<64>::kAlloc, st>>>(p);
-    }
-    return launched();
+    return run_scores(L, q, k, stats, scores, status, st);
 }
 
 extern "C" spava_status spava_score_noalloc_status(void *stream, int32_t *flags) {

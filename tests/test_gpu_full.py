@@ -75,6 +75,14 @@ def test_full_size_layer(name):
         np.testing.assert_allclose(sc[g, :last0], sc_ref[g, :last0], rtol=SCORE_REL,
                                    atol=1e-7 * w.q * w.Hq / w.Hkv)
     rep = check_selection(w, sc_ref, idx_h, groups, idx_ref)
+    # Every selection of every KV group is, bit for bit, the top-l of the GPU's
+    # own fp32 scores (ties to the lower index): the selection step is exact
+    # even where the oracle's fp64 scores leave a band of valid choices.
+    for u in range(2 * w.H - 1):
+        s0, n = int(off[u] - w.a), int(off[u + 1] - off[u])
+        for g in range(w.Hkv):
+            want = oracle.select_top_l(sc[g, s0:s0 + n].astype(np.float64), int(off[u]), w.l)
+            np.testing.assert_array_equal(idx_h[u, g], want, err_msg=f"{name} u={u} g={g}")
 
     # Every sampled row and head against the oracle's attention over the key
     # sets of the GPU's (accepted) selection: nothing is exempt.
