@@ -337,6 +337,7 @@ struct FusedSelect {
     const void *v;
     void *pk, *pv;
     int *counters;
+    bool anchor;  // also copy the anchor rows into the packed buffers
 };
 
 // Query-to-context scores of the producing chunks held here, normalised by
@@ -370,7 +371,7 @@ spava_status run_scores(const Layer &L, const void *q, const void *k, const floa
         p.PK = static_cast<__nv_bfloat16 *>(fused->pk);
         p.PV = static_cast<__nv_bfloat16 *>(fused->pv);
         p.n_score_ctas = static_cast<int32_t>(score_ctas);
-        blocks += L.a > 0 ? static_cast<int64_t>(L.Hkv) * cdiv(L.a, kAnchorRowsPerCta) : 0;
+        if (fused->anchor && L.a > 0) blocks += static_cast<int64_t>(L.Hkv) * cdiv(L.a, kAnchorRowsPerCta);
         SPAVA_CUDA(cudaMemsetAsync(p.counters, 0, sizeof(int32_t) * size_t(L.n_chunks - 1) * L.Hkv, st));
     }
     if (blocks == 0) return SPAVA_OK;
@@ -390,11 +391,12 @@ spava_status run_scores(const Layer &L, const void *q, const void *k, const floa
 // The same, with the workspace's status word and counters.
 spava_status run_scores_ws(const Layer &L, const void *q, const void *k, const float *stats, float *scores,
                            char *ws, cudaStream_t st, bool fused = false, int32_t *idx = nullptr,
-                           const void *v = nullptr, void *pk = nullptr, void *pv = nullptr) {
+                           const void *v = nullptr, void *pk = nullptr, void *pv = nullptr,
+                           bool anchor = true) {
     const WsLayout w = ws_layout(L);
     int *status = reinterpret_cast<int *>(ws + w.status);
     if (!fused) return run_scores(L, q, k, stats, scores, status, st);
-    const FusedSelect f{idx, v, pk, pv, reinterpret_cast<int *>(ws + w.counters)};
+    const FusedSelect f{idx, v, pk, pv, reinterpret_cast<int *>(ws + w.counters), anchor};
     return run_scores(L, q, k, stats, scores, status, st, &f);
 }
 
@@ -713,57 +715,146 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
                                           ws_bytes, stream));
         return d2h_rows(0, L.N, st);
     }
-    // Pipelined: K and the query block's Q rows (all that scoring needs) go up
-    // first, then V (the gather needs it), then the Q rows of each context
-    // group; the attention runs group by group as its Q rows arrive, and each
-    // group's O goes down while later groups compute.  The copies start only
-    // once everything already on `stream` is done (an earlier call's kernels may
-    // still be reading the device buffers they overwrite).
     cudaStream_t cs = static_cast<cudaStream_t>(copy_stream);
-    int lo[kCopyGroups], hi[kCopyGroups];
-    const int ng = copy_groups(L, lo, hi);
-    // start, front, V, Q of groups 1.., attention of each group, done
-    std::vector<cudaEvent_t> ev(2 * ng + 4, nullptr);
+    char *w = static_cast<char *>(ws);
+    const WsLayout lay = ws_layout(L);
+    auto cv = static_cast<const char *>(v_host), ck = static_cast<const char *>(k_host);
+    char *kd = static_cast<char *>(k), *vd = static_cast<char *>(v);
+    auto h2d_rows = [&](int r0, int r1, bool qkv) -> spava_status {  // Q rows, and K/V rows if qkv
+        if (r1 <= r0) return SPAVA_OK;
+        SPAVA_CUDA(cudaMemcpyAsync(qd + r0 * row_q, cq + r0 * row_q, (r1 - r0) * row_q,
+                                   cudaMemcpyHostToDevice, cs));
+        if (qkv) {
+            SPAVA_CUDA(cudaMemcpyAsync(kd + r0 * row_k, ck + r0 * row_k, (r1 - r0) * row_k,
+                                       cudaMemcpyHostToDevice, cs));
+            SPAVA_CUDA(cudaMemcpyAsync(vd + r0 * row_k, cv + r0 * row_k, (r1 - r0) * row_k,
+                                       cudaMemcpyHostToDevice, cs));
+        }
+        return SPAVA_OK;
+    };
+    std::vector<cudaEvent_t> ev;
     spava_status rc = SPAVA_OK;
-    for (auto &e : ev)
+    auto new_event = [&]() -> cudaEvent_t {
+        cudaEvent_t e = nullptr;
         if (rc == SPAVA_OK && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
             rc = cuda_fail(cudaGetLastError());
+        ev.push_back(e);
+        return e;
+    };
+    const bool chunkwise = L.norm == 0;
     auto body = [&]() -> spava_status {
-        cudaEvent_t e_start = ev[0], e_front = ev[1], e_v = ev[2], *e_q = &ev[3], *e_a = &ev[3 + ng],
-                    e_done = ev[3 + 2 * ng];
+        cudaEvent_t e_start = new_event();
+        if (rc != SPAVA_OK) return rc;
+        // The copies start only once everything already on `stream` is done (an
+        // earlier call's kernels may still be reading the buffers they overwrite).
         SPAVA_CUDA(cudaEventRecord(e_start, st));
         SPAVA_CUDA(cudaStreamWaitEvent(cs, e_start, 0));
-        SPAVA_CUDA(cudaMemcpyAsync(k, k_host, L.N * row_k, cudaMemcpyHostToDevice, cs));
-        SPAVA_CUDA(cudaMemcpyAsync(qd + lo[0] * row_q, cq + lo[0] * row_q, (hi[0] - lo[0]) * row_q,
-                                   cudaMemcpyHostToDevice, cs));
-        SPAVA_CUDA(cudaEventRecord(e_front, cs));
-        SPAVA_CUDA(cudaMemcpyAsync(v, v_host, L.N * row_k, cudaMemcpyHostToDevice, cs));
-        SPAVA_CUDA(cudaEventRecord(e_v, cs));
-        for (int g = 1; g < ng; ++g) {
-            SPAVA_CUDA(cudaMemcpyAsync(qd + lo[g] * row_q, cq + lo[g] * row_q, (hi[g] - lo[g]) * row_q,
-                                       cudaMemcpyHostToDevice, cs));
-            SPAVA_CUDA(cudaEventRecord(e_q[g], cs));
+        std::vector<std::pair<int, int>> rows;      // row groups, in the order they compute
+        std::vector<cudaEvent_t> computed;          // one per row group
+        if (chunkwise) {
+            // Chunk by chunk, in token order: chunk v's rows need the anchor, the
+            // passing blocks of the chunks before it, its partner chunk (an
+            // earlier one) and itself -- all on the device by the time chunk v
+            // has arrived -- so each chunk is scored, selected and gathered, and
+            // its rows computed, as soon as its Q/K/V rows land, while the next
+            // chunk is still on its way.  The query block's Q rows (the scorer)
+            // go up first, its K/V last; its rows compute last.
+            const int q0 = L.N - L.q;
+            SPAVA_TRY(h2d_rows(q0, L.N, false));
+            SPAVA_TRY(h2d_rows(0, L.a, true));
+            cudaEvent_t e_anchor = new_event();
+            std::vector<cudaEvent_t> e_chunk(L.n_chunks);
+            for (auto &e : e_chunk) e = new_event();
+            cudaEvent_t e_query = new_event();
+            if (rc != SPAVA_OK) return rc;
+            SPAVA_CUDA(cudaEventRecord(e_anchor, cs));
+            for (int c = 0; c < L.n_chunks; ++c) {
+                SPAVA_TRY(h2d_rows(L.off[c], L.off[c + 1], true));
+                SPAVA_CUDA(cudaEventRecord(e_chunk[c], cs));
+            }
+            SPAVA_CUDA(cudaMemcpyAsync(kd + q0 * row_k, ck + q0 * row_k, L.q * row_k, cudaMemcpyHostToDevice, cs));
+            SPAVA_CUDA(cudaMemcpyAsync(vd + q0 * row_k, cv + q0 * row_k, L.q * row_k, cudaMemcpyHostToDevice, cs));
+            SPAVA_CUDA(cudaEventRecord(e_query, cs));
+            const bool select = L.n_chunks > 1 && L.l > 0;
+            float *scores = reinterpret_cast<float *>(w + lay.scores);
+            const float *stats = reinterpret_cast<const float *>(w + lay.stats);
+            int32_t *idx = reinterpret_cast<int32_t *>(w + lay.idx);
+            SPAVA_CUDA(cudaStreamWaitEvent(st, e_anchor, 0));
+            if (!select) SPAVA_TRY(run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st));  // anchor rows
+            auto attend = [&](int r0, int r1) -> spava_status {
+                if (r1 <= r0) return SPAVA_OK;
+                SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, want_lse ? lse : nullptr, w, st,
+                                   r0, r1));
+                cudaEvent_t e = new_event();
+                if (rc != SPAVA_OK) return rc;
+                SPAVA_CUDA(cudaEventRecord(e, st));
+                rows.emplace_back(r0, r1);
+                computed.push_back(e);
+                return SPAVA_OK;
+            };
+            SPAVA_TRY(attend(0, L.a));
+            for (int c = 0; c < L.n_chunks; ++c) {
+                SPAVA_CUDA(cudaStreamWaitEvent(st, e_chunk[c], 0));
+                if (select && c < L.n_chunks - 1) {
+                    // this chunk's passing block: the same kernels as the whole
+                    // layer's front, restricted to chunk c
+                    Layer Lc = L;
+                    Lc.own = 1ULL << c;
+                    SPAVA_TRY(run_stats(Lc, q, k, w, st));
+                    SPAVA_TRY(run_scores_ws(Lc, q, k, stats, scores, w, st, true, idx, v, w + lay.pk,
+                                            w + lay.pv, c == 0));
+                }
+                SPAVA_TRY(attend(L.off[c], L.off[c + 1]));
+            }
+            SPAVA_CUDA(cudaStreamWaitEvent(st, e_query, 0));
+            SPAVA_TRY(attend(q0, L.N));
+        } else {
+            // Row-normalised scores need every segment's statistics first: K and
+            // the query block's Q rows go up first, then V, then the Q rows of
+            // each context group; the attention runs group by group as its Q rows
+            // arrive.
+            int lo[kCopyGroups], hi[kCopyGroups];
+            const int ng = copy_groups(L, lo, hi);
+            cudaEvent_t e_front = new_event(), e_v = new_event();
+            std::vector<cudaEvent_t> e_q(ng);
+            for (auto &e : e_q) e = new_event();
+            if (rc != SPAVA_OK) return rc;
+            SPAVA_CUDA(cudaMemcpyAsync(k, k_host, L.N * row_k, cudaMemcpyHostToDevice, cs));
+            SPAVA_TRY(h2d_rows(lo[0], hi[0], false));
+            SPAVA_CUDA(cudaEventRecord(e_front, cs));
+            SPAVA_CUDA(cudaMemcpyAsync(v, v_host, L.N * row_k, cudaMemcpyHostToDevice, cs));
+            SPAVA_CUDA(cudaEventRecord(e_v, cs));
+            for (int g = 1; g < ng; ++g) {
+                SPAVA_TRY(h2d_rows(lo[g], hi[g], false));
+                SPAVA_CUDA(cudaEventRecord(e_q[g], cs));
+            }
+            SPAVA_CUDA(cudaStreamWaitEvent(st, e_front, 0));
+            SPAVA_TRY(run_front(L, q, k, v, nullptr, w, st, e_v));
+            for (int g = 0; g < ng; ++g) {
+                if (g > 0) SPAVA_CUDA(cudaStreamWaitEvent(st, e_q[g], 0));
+                SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, want_lse ? lse : nullptr, w,
+                                   st, lo[g], hi[g]));
+                cudaEvent_t e = new_event();
+                if (rc != SPAVA_OK) return rc;
+                SPAVA_CUDA(cudaEventRecord(e, st));
+                rows.emplace_back(lo[g], hi[g]);
+                computed.push_back(e);
+            }
         }
-        char *w = static_cast<char *>(ws);
-        const WsLayout lay = ws_layout(L);
-        SPAVA_CUDA(cudaStreamWaitEvent(st, e_front, 0));
-        SPAVA_TRY(run_front(L, q, k, v, nullptr, w, st, e_v));
-        for (int g = 0; g < ng; ++g) {
-            if (g > 0) SPAVA_CUDA(cudaStreamWaitEvent(st, e_q[g], 0));
-            SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, want_lse ? lse : nullptr, w,
-                               st, lo[g], hi[g]));
-            SPAVA_CUDA(cudaEventRecord(e_a[g], st));
-        }
-        for (int g = 0; g < ng; ++g) {
-            SPAVA_CUDA(cudaStreamWaitEvent(cs, e_a[g], 0));
-            SPAVA_TRY(d2h_rows(lo[g], hi[g], cs));
+        // Each row group's O (and lse) goes down once it is computed.
+        for (size_t g = 0; g < rows.size(); ++g) {
+            SPAVA_CUDA(cudaStreamWaitEvent(cs, computed[g], 0));
+            SPAVA_TRY(d2h_rows(rows[g].first, rows[g].second, cs));
         }
         // The call's work ends on `stream`, after the last copy.
+        cudaEvent_t e_done = new_event();
+        if (rc != SPAVA_OK) return rc;
         SPAVA_CUDA(cudaEventRecord(e_done, cs));
         SPAVA_CUDA(cudaStreamWaitEvent(st, e_done, 0));
         return SPAVA_OK;
     };
-    if (rc == SPAVA_OK) rc = body();
+    const spava_status rb = body();
+    if (rc == SPAVA_OK) rc = rb;
     // Destroying a recorded event is safe: its resources go once it completes.
     for (auto e : ev)
         if (e) cudaEventDestroy(e);
