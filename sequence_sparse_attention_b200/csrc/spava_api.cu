@@ -28,6 +28,8 @@ spava_status cuda_fail(cudaError_t e) {
     return SPAVA_ERR_CUDA;
 }
 
+spava_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? SPAVA_OK : cuda_fail(e); }
+
 #define SPAVA_CUDA(...)                                    \
     do {                                                   \
         cudaError_t e_ = (__VA_ARGS__);                           \
@@ -775,10 +777,30 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
             SPAVA_CUDA(cudaMemcpyAsync(kd + q0 * row_k, ck + q0 * row_k, L.q * row_k, cudaMemcpyHostToDevice, cs));
             SPAVA_CUDA(cudaMemcpyAsync(vd + q0 * row_k, cv + q0 * row_k, L.q * row_k, cudaMemcpyHostToDevice, cs));
             SPAVA_CUDA(cudaEventRecord(e_query, cs));
+            // A region's last 128-row tile reads up to 127 rows past the region's
+            // end: their keys are masked, but their V rows meet a zero weight in
+            // the PV product, and 0 x (a NaN or Inf not yet overwritten) is NaN.
+            // So a region's attention waits until every row its tiles touch has
+            // arrived.
+            auto wait_rows = [&](int end) -> spava_status {  // rows [0, end) on the device
+                if (end > L.off[L.n_chunks]) return cuda_ok(cudaStreamWaitEvent(st, e_query, 0));
+                int c = 0;
+                while (L.off[c + 1] < end) ++c;
+                return cuda_ok(cudaStreamWaitEvent(st, e_chunk[c], 0));
+            };
+            auto tiles_end = [&](int r0, int r1) { return std::min(L.N, r0 + kRowTile * cdiv(r1 - r0, kRowTile)); };
             const bool select = L.n_chunks > 1 && L.l > 0;
             float *scores = reinterpret_cast<float *>(w + lay.scores);
             const float *stats = reinterpret_cast<const float *>(w + lay.stats);
             int32_t *idx = reinterpret_cast<int32_t *>(w + lay.idx);
+            // The packed passing blocks fill up chunk by chunk, and a packed
+            // segment's last tile reads past its end into blocks not yet written:
+            // those rows start as zeros, not as whatever the workspace held.
+            if (select) {
+                const size_t packed = 2 * size_t(L.Hkv) * L.L * L.d;
+                SPAVA_CUDA(cudaMemsetAsync(w + lay.pk, 0, packed, st));
+                SPAVA_CUDA(cudaMemsetAsync(w + lay.pv, 0, packed, st));
+            }
             SPAVA_CUDA(cudaStreamWaitEvent(st, e_anchor, 0));
             if (!select) SPAVA_TRY(run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st));  // anchor rows
             auto attend = [&](int r0, int r1) -> spava_status {
@@ -792,7 +814,10 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
                 computed.push_back(e);
                 return SPAVA_OK;
             };
-            SPAVA_TRY(attend(0, L.a));
+            if (L.a > 0) {
+                SPAVA_TRY(wait_rows(tiles_end(0, L.a)));
+                SPAVA_TRY(attend(0, L.a));
+            }
             for (int c = 0; c < L.n_chunks; ++c) {
                 SPAVA_CUDA(cudaStreamWaitEvent(st, e_chunk[c], 0));
                 if (select && c < L.n_chunks - 1) {
@@ -804,6 +829,7 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
                     SPAVA_TRY(run_scores_ws(Lc, q, k, stats, scores, w, st, true, idx, v, w + lay.pk,
                                             w + lay.pv, c == 0));
                 }
+                SPAVA_TRY(wait_rows(tiles_end(L.off[c], L.off[c + 1])));
                 SPAVA_TRY(attend(L.off[c], L.off[c + 1]));
             }
             SPAVA_CUDA(cudaStreamWaitEvent(st, e_query, 0));

@@ -230,8 +230,10 @@ def test_host_buffers_entry_point(name, pipelined):
     qh, kh, vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
     oh = torch.full_like(Q, 7.0).pin_memory()
     lh = torch.full((w.Hq, w.N), 7.0, dtype=torch.float32).pin_memory()
-    qd, kd, vd = torch.empty_like(Q, device="cuda"), torch.empty_like(K, device="cuda"), torch.empty_like(V, device="cuda")
-    od = torch.empty_like(qd)
+    # device buffers start as NaN: a kernel that read a row before its upload
+    # landed would show it
+    qd, kd, vd = (torch.full_like(x, float("nan"), device="cuda") for x in (Q, K, V))
+    od = torch.full_like(qd, float("nan"))
     ld = torch.empty((w.Hq, w.N), dtype=torch.float32, device="cuda")
     cs = torch.cuda.Stream() if pipelined else None
     sp.prefill_attention_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, copy_stream=cs)
@@ -251,10 +253,10 @@ def test_host_buffers_back_to_back():
     w = WORKLOADS["16k"]
     ins = [make_inputs(w), make_inputs(dataclasses.replace(w, seed=w.seed + 100))]
     sp = Spava(Layout.from_workload(w))
-    qd = torch.empty(ins[0][0].shape, dtype=torch.bfloat16, device="cuda")
-    kd = torch.empty(ins[0][1].shape, dtype=torch.bfloat16, device="cuda")
-    vd = torch.empty_like(kd)
-    od = torch.empty_like(qd)
+    qd = torch.full(ins[0][0].shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    kd = torch.full(ins[0][1].shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    vd = torch.full_like(kd, float("nan"))
+    od = torch.full_like(qd, float("nan"))
     cs = torch.cuda.Stream()
     outs = []
     hosts = []
