@@ -140,9 +140,14 @@ spava_status spava_attn(const spava_config *cfg, const void *q, const void *k, c
                         const void *pk, const void *pv, void *o, float *lse, void *ws,
                         size_t ws_bytes, void *stream);
 
-/* The whole layer: spava_score -> spava_topk_select -> spava_pack_passing ->
- * spava_attn, with scores, idx and the packed K/V kept in the workspace.  If
- * idx_out != NULL the passing-block indices are also written there. */
+/* The whole layer, in the order of the fused forward ("Forward Fuso di
+ * Contesto e Query"): first the anchor rows and the query rows' per-segment
+ * partials, whose per-chunk log-sum-exps are the scoring's normaliser; then
+ * scoring, selection and gather of every passing block in one launch; then the
+ * context rows and the query-row merge.  Scores, idx and the packed K/V stay in
+ * the workspace.  The outputs equal, byte for byte, those of spava_score ->
+ * spava_topk_select -> spava_pack_passing -> spava_attn.  If idx_out != NULL
+ * the passing-block indices are also written there. */
 spava_status spava_prefill_attention(const spava_config *cfg, const void *q, const void *k,
                                      const void *v, void *o, float *lse, int32_t *idx_out,
                                      void *ws, size_t ws_bytes, void *stream);
@@ -154,11 +159,15 @@ spava_status spava_prefill_attention(const spava_config *cfg, const void *q, con
  * call does not wait for them.
  * copy_stream NULL (or equal to stream): everything is ordered on `stream`.
  * Otherwise the copies run on copy_stream, overlapped with the kernels on
- * `stream`: K and the query block's Q rows go up first (all that scoring
- * needs), then V; the attention then runs in up to 8 groups of whole regions
- * (the query block, then chunks and anchor in descending token order, costliest
- * first), each starting once its Q rows have arrived, and each group's O (and
- * lse) rows go down while later groups compute.  The copies begin only after
+ * `stream`, chunk by chunk in token order: the query block's Q rows and the
+ * anchor go up first, then each chunk's Q, K and V rows; once a chunk (and the
+ * rows its last 128-row tile reaches into) has arrived, its passing block is
+ * scored, selected and gathered and its rows are computed, and its O (and lse)
+ * rows go down while later chunks compute; the query block's rows come last.
+ * (With score_norm 1 -- whose statistics need every segment first -- K and the
+ * query block's Q rows go up first, then V, and the attention runs in up to 8
+ * groups of whole regions as their Q rows arrive.)  The outputs equal
+ * spava_prefill_attention's byte for byte.  The copies begin only after
  * all work already enqueued on `stream` (an earlier call may still be reading
  * the device buffers), and `stream` is made to wait for the last copy, so the
  * call's work is complete when `stream` is and back-to-back calls on the same
