@@ -271,26 +271,28 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const Layer L, const
         // Source element offset of this lane's row, or -1 (past the end, or an
         // index that is not a token position: written as a zero row).
         const long long row_l = grp * 32 + lane;
-        long long src_l = -2;
+        long long src_l = -1;
+        int src = -2;
         if (row_l < total) {
             const int g = static_cast<int>(row_l / L.L);
-            const int src = packed_source(L, idx, g, static_cast<int>(row_l % L.L));
-            src_l = src >= 0 ? (static_cast<long long>(src) * L.Hkv + g) * D : src;
+            src = packed_source(L, idx, g, static_cast<int>(row_l % L.L));
+            if (src >= 0) src_l = (static_cast<long long>(src) * L.Hkv + g) * D;
         }
+        // rows to leave alone: past the end, or of a chunk not held here
+        const uint32_t keep = __ballot_sync(0xffffffffu, src != -2);
 #pragma unroll 1
         for (int b = 0; b < 32; b += kPackBatch) {
             uint4 v[kPackBatch];
-            long long so[kPackBatch];
 #pragma unroll
             for (int k = 0; k < kPackBatch; ++k) {
-                so[k] = __shfl_sync(0xffffffffu, src_l, b + k);
+                const long long so = __shfl_sync(0xffffffffu, src_l, b + k);
                 v[k] = make_uint4(0, 0, 0, 0);
-                if (so[k] >= 0 && c < kChunks) v[k] = __ldg(reinterpret_cast<const uint4 *>(src_base + so[k]) + c);
+                if (so >= 0 && c < kChunks) v[k] = __ldg(reinterpret_cast<const uint4 *>(src_base + so) + c);
             }
 #pragma unroll
             for (int k = 0; k < kPackBatch; ++k) {
                 const long long row = grp * 32 + b + k;
-                if (row < total && so[k] != -2 && c < kChunks)
+                if (((keep >> (b + k)) & 1u) && c < kChunks)
                     reinterpret_cast<uint4 *>(dst_base + row * D)[c] = v[k];
             }
         }
