@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
     SPAVA_OK = 0,
     SPAVA_ERR_INVALID_ARG = 1, /* a size, offset or pointer is invalid */
-    SPAVA_ERR_UNSUPPORTED = 2, /* valid, but outside what this build runs (d, H) */
+    SPAVA_ERR_UNSUPPORTED = 2, /* valid, but outside what the library supports (d, H, ...) */
     SPAVA_ERR_MISALIGNED = 3,  /* a device pointer is not 16-byte aligned */
     SPAVA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
     SPAVA_ERR_CUDA = 5,        /* a CUDA runtime call failed */
