@@ -60,6 +60,12 @@ CASES = {
                          seed=26, local_pair_full=0),
     "variants_d64": Workload("variants_d64", H=3, Hq=6, Hkv=3, d=64, N=1500, a=64, q=140, l=50,
                              frame=32, seed=27, score_norm=1, score_pool=3),
+    # the most hosts the library takes (H = 32: 64 chunks, a full 64-bit host mask)
+    "max_hosts": Workload("max_hosts", H=32, Hq=4, Hkv=2, d=64, N=64 + 64 * 41 + 40, a=64, q=40, l=16,
+                          frame=16, seed=29),
+    # the smallest query block and anchor: one row each
+    "one_row_query": Workload("one_row_query", H=2, Hq=4, Hkv=2, d=128, N=1 + 4 * 200 + 1, a=1, q=1,
+                              l=50, frame=16, seed=30),
 }
 
 

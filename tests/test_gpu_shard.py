@@ -26,6 +26,8 @@ CASES = {
                        frame=32, seed=35, score_pool=5),
     "heavy_jitter": Workload("heavy_jitter", H=4, Hq=4, Hkv=1, d=128, N=80 + 64 * 40 + 60, a=80, q=60,
                              l=70, frame=64, jitter=0.1, heavy_frac=0.05, seed=36),
+    "max_hosts": Workload("max_hosts", H=32, Hq=4, Hkv=2, d=64, N=64 + 64 * 41 + 40, a=64, q=40, l=16,
+                          frame=16, seed=37),
 }
 
 
