@@ -69,9 +69,9 @@ __host__ __device__ inline int query_region(const Layer &L) { return L.n_chunks 
 __host__ __device__ inline bool owns(const Layer &L, int v) { return (L.own >> v) & 1u; }
 
 // A run of work items of one kind and one chunk/segment.  Items inside a group
-// are ordered (KV head, row tile descending, query head of that KV head): the
+// run KV head by KV head, the costlier row tiles first (decode_pair_item): the
 // CTAs resident at any moment then work on one KV head's packed passing K/V and
-// chunks, which fit in L2, and within a KV head the costlier row tiles go first.
+// chunks, which fit in L2.
 struct Group {
     int32_t kind, sub, n_rt, item_begin;
 };
@@ -88,22 +88,6 @@ struct Seg {
 __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 __host__ __device__ inline int pair_of(int H, int v) { return v < H ? v : 2 * H - 1 - v; }
-
-__host__ __device__ inline Item decode_item(const Group *groups, int n_groups, int b, int Hq,
-                                            int G) {
-    int k = 0;
-    while (k + 1 < n_groups && b >= groups[k + 1].item_begin) ++k;
-    const Group &g = groups[k];
-    const int i = b - g.item_begin;
-    const int per_kv = g.n_rt * G;  // items of one KV head
-    const int rem = i % per_kv;
-    Item it;
-    it.kind = g.kind;
-    it.sub = g.sub;
-    it.rt = g.n_rt - 1 - rem / G;
-    it.h = (i / per_kv) * G + rem % G;
-    return it;
-}
 
 // Rows [row0, row_end) of the item.
 __host__ __device__ inline void item_rows(const Layer &L, const Item &it, int &row0, int &row_end) {

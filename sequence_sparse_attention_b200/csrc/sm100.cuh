@@ -250,19 +250,6 @@ __device__ __forceinline__ void reg_dealloc() {
 __device__ __forceinline__ void bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-// Named barrier that also ANDs a predicate over its participants: every
-// participant gets the same answer, so they can leave a loop together.
-__device__ __forceinline__ bool bar_red_and(int id, int n, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
-        : "=r"(r)
-        : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
-        : "memory");
-    return r != 0;
-}
-
 // ------------------------------------------------------------------ math
 // Hardware base-2 exponential (MUFU.EX2), flush-to-zero approximate.
 __device__ __forceinline__ float ex2(float x) {
@@ -295,20 +282,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
-// Max of 64 values with 4 independent chains of 3-input max.
-__device__ __forceinline__ float max64(const float (&x)[64]) {
-    float m[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) m[k] = x[k];
-#pragma unroll
-    for (int c = 4; c + 8 <= 64; c += 8)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) m[k] = fmax3(m[k], x[c + k], x[c + 4 + k]);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], x[60 + k]);
-    return fmaxf(fmax3(m[0], m[1], m[2]), m[3]);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
     return *reinterpret_cast<uint32_t *>(&v);

@@ -115,7 +115,7 @@ void region_rows(const Layer &L, int kind, int sub, int &lo, int &hi) {
 // order), so a cost-descending order is a longest-processing-time-first
 // schedule over the SMs.  Inside a group, items run KV head by KV head, row
 // tile descending, with the query heads of a KV head adjacent (shared K/V tiles
-// in L2; see decode_pair_item and decode_item).  Only regions lying inside
+// in L2; see decode_pair_item).  Only regions lying inside
 // rows [row_lo, row_hi) are planned (the whole layer by default).
 constexpr unsigned kAllKinds = (1u << kCtx) | (1u << kAnchor) | (1u << kQueryPart);
 int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int row_hi = INT32_MAX,
@@ -161,7 +161,7 @@ int plan_attention(const Layer &L, bool stats, Group *out, int row_lo = 0, int r
     return n;
 }
 
-int64_t plan_items(const Group *g, int n, const Layer &L, bool /*stats*/) {
+int64_t plan_items(const Group *g, int n, const Layer &L) {
     if (!n) return 0;
     return static_cast<int64_t>(g[n - 1].item_begin) + pair_items(g[n - 1].n_rt, L.G) * L.Hkv;
 }
@@ -270,7 +270,7 @@ spava_status launched() {
 // ---------------------------------------------------------------- launches
 template <int D, bool STATS>
 spava_status launch_attn(AttnParams &p, cudaStream_t st) {
-    const int64_t items = plan_items(p.groups, p.n_groups, p.L, false);
+    const int64_t items = plan_items(p.groups, p.n_groups, p.L);
     if (items == 0) return SPAVA_OK;
     if (items >= (1LL << 31)) return SPAVA_ERR_UNSUPPORTED;
     using SM = AttnSmem<D>;
@@ -1125,9 +1125,6 @@ spava_status part_slot_copy(Copier &cp, const Layer &L, char *ws, char *msg, con
     return SPAVA_OK;
 }
 
-spava_status check_shard_args(const Layer &L, void *ws, size_t ws_bytes) {
-    return check_ws(L, ws, ws_bytes);
-}
 
 }  // namespace
 
@@ -1167,7 +1164,7 @@ spava_status spava_shard_front(const spava_config *cfg, int32_t rank, int32_t wo
     SPAVA_TRY(check_ptr(k));
     SPAVA_TRY(check_ptr(v));
     SPAVA_TRY(check_ptr(pass_send));
-    SPAVA_TRY(check_shard_args(L, ws, ws_bytes));
+    SPAVA_TRY(check_ws(L, ws, ws_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *w = static_cast<char *>(ws);
     SPAVA_TRY(run_front(L, q, k, v, nullptr, w, st));
@@ -1191,7 +1188,7 @@ spava_status spava_shard_local_attn(const spava_config *cfg, int32_t rank, int32
     SPAVA_TRY(check_ptr(o));
     SPAVA_TRY(check_ptr(lse, false));
     SPAVA_TRY(check_ptr(part_send));
-    SPAVA_TRY(check_shard_args(L, ws, ws_bytes));
+    SPAVA_TRY(check_ws(L, ws, ws_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *w = static_cast<char *>(ws);
     const WsLayout lay = ws_layout(L);
@@ -1221,7 +1218,7 @@ spava_status spava_shard_context_attn(const spava_config *cfg, int32_t rank, int
     SPAVA_TRY(check_ptr(lse, false));
     SPAVA_TRY(check_ptr(pass_all));
     SPAVA_TRY(check_ptr(idx_out, false));
-    SPAVA_TRY(check_shard_args(L, ws, ws_bytes));
+    SPAVA_TRY(check_ws(L, ws, ws_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *w = static_cast<char *>(ws);
     const WsLayout lay = ws_layout(L);
@@ -1252,7 +1249,7 @@ spava_status spava_shard_merge(const spava_config *cfg, int32_t rank, int32_t wo
     SPAVA_TRY(check_ptr(o));
     SPAVA_TRY(check_ptr(lse, false));
     SPAVA_TRY(check_ptr(part_all));
-    SPAVA_TRY(check_shard_args(L, ws, ws_bytes));
+    SPAVA_TRY(check_ws(L, ws, ws_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *w = static_cast<char *>(ws);
     const PartMsg g = part_msg(L, world);
