@@ -185,3 +185,35 @@ def test_two_gloo_ranks_exchange_what_their_rows_need():
         assert same_idx, f"rank {rank}: gathered selection differs from the oracle's"
         assert exact, f"rank {rank}: its rows need data it neither holds nor received"
         assert segs == list(range(1, 2 * W.H + 1))       # every chunk's partial exactly once
+
+
+def test_shard_calls_reject_bad_arguments_before_any_launch():
+    """Missing or misaligned pointers and a missing or misaligned workspace are
+    refused by every shard call before anything is launched (no GPU needed)."""
+    lay = Layout.from_workload(WORKLOADS["16k"])
+    cfg = lay.c()
+    lib = native.load()
+    ws_b, _, _ = shard_sizes(lay, 2)
+    good = 1 << 20          # an aligned, never dereferenced address
+    odd = good + 8          # 16-byte misaligned
+    ws = 1 << 24            # 256-byte aligned
+    c = ctypes.byref(cfg)
+    # front: q, k, v, pass_send, ws
+    assert lib.spava_shard_front(c, 0, 2, None, good, good, good, ws, ws_b, None) == 1
+    assert lib.spava_shard_front(c, 0, 2, good, good, good, odd, ws, ws_b, None) == 3
+    assert lib.spava_shard_front(c, 0, 2, good, good, good, good, None, ws_b, None) == 4
+    assert lib.spava_shard_front(c, 0, 2, good, good, good, good, ws + 16, ws_b, None) == 3
+    assert lib.spava_shard_front(c, 0, 2, good, good, good, good, ws, ws_b - 256, None) == 4
+    assert lib.spava_shard_front(c, 2, 2, good, good, good, good, ws, ws_b, None) == 1
+    # local attention: o, lse (optional), part_send
+    assert lib.spava_shard_local_attn(c, 1, 2, good, good, good, None, None, good, ws, ws_b, None) == 1
+    assert lib.spava_shard_local_attn(c, 1, 2, good, good, good, good, odd, good, ws, ws_b, None) == 3
+    # context attention: pass_all required, idx_out optional but aligned
+    assert lib.spava_shard_context_attn(c, 0, 2, good, good, good, None, good, None, None, ws, ws_b, None) == 1
+    assert lib.spava_shard_context_attn(c, 0, 2, good, good, good, good, good, None, odd, ws, ws_b, None) == 3
+    # merge: part_all required
+    assert lib.spava_shard_merge(c, 0, 2, None, good, None, ws, ws_b, None) == 1
+
+
+def test_noalloc_status_rejects_a_missing_output():
+    assert native.load().spava_score_noalloc_status(None, None) == 1
