@@ -158,12 +158,17 @@ spava_status spava_prefill_attention(const spava_config *cfg, const void *q, con
  * Host buffers should be page-locked for the copies to be asynchronous; the
  * call does not wait for them.
  * copy_stream NULL (or equal to stream): everything is ordered on `stream`.
- * Otherwise the copies run on copy_stream, overlapped with the kernels on
- * `stream`, chunk by chunk in token order: the query block's Q rows and the
- * anchor go up first, then each chunk's Q, K and V rows; once a chunk (and the
- * rows its last 128-row tile reaches into) has arrived, its passing block is
- * scored, selected and gathered and its rows are computed, and its O (and lse)
- * rows go down while later chunks compute; the query block's rows come last.
+ * Otherwise the copies run on copy_stream, overlapped with the kernels,
+ * chunk by chunk in token order: the query block's Q rows and the anchor go up
+ * first, then each chunk's Q, K and V rows; once a chunk (and the rows its last
+ * 128-row tile reaches into) has arrived, its passing block is scored, selected
+ * and gathered and its rows are computed, and its O (and lse) rows go down
+ * while later chunks compute; the query block's rows come last.  The kernels
+ * of this mode run on three streams the call creates and destroys: scoring at
+ * the device's highest stream priority, and the attention launches alternating
+ * between two others, each launch waiting only for its rows and the passing
+ * blocks before them, so that one launch's CTAs take the SMs its
+ * predecessor's last work items leave idle.
  * (With score_norm 1 -- whose statistics need every segment first -- K and the
  * query block's Q rows go up first, then V, and the attention runs in up to 8
  * groups of whole regions as their Q rows arrive.)  The outputs equal
@@ -171,8 +176,8 @@ spava_status spava_prefill_attention(const spava_config *cfg, const void *q, con
  * all work already enqueued on `stream` (an earlier call may still be reading
  * the device buffers), and `stream` is made to wait for the last copy, so the
  * call's work is complete when `stream` is and back-to-back calls on the same
- * buffers stay ordered.  The call creates and destroys its own CUDA events (no
- * memory).  Neither stream may be capturing a graph.  On an error return, work
+ * buffers stay ordered.  The call creates and destroys its own CUDA events
+ * and streams (no memory).  Neither stream may be capturing a graph.  On an error return, work
  * already enqueued may still run. */
 spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q_host,
                                           const void *k_host, const void *v_host, void *o_host,

@@ -197,6 +197,12 @@ spava_status check_ws(const Layer &L, void *ws, size_t ws_bytes) {
     return SPAVA_OK;
 }
 
+// Work-queue counters of the persistent attention launches, inside the
+// workspace's first 256 bytes (the status block: status word at 0): slot 0
+// serves every launch on the caller's stream and the statistics pass; launches
+// that may run at the same time as another attention launch take slots 1 and 2.
+int *queue_slot(char *ws, int slot) { return reinterpret_cast<int *>(ws + 128 + 32 * slot); }
+
 spava_status check_ptr(const void *p, bool required = true) {
     if (!p) return required ? SPAVA_ERR_INVALID_ARG : SPAVA_OK;
     return (reinterpret_cast<uintptr_t>(p) & 15) ? SPAVA_ERR_MISALIGNED : SPAVA_OK;
@@ -308,7 +314,7 @@ spava_status run_stats(const Layer &L, const void *q, const void *k, char *ws, c
     float *stats = reinterpret_cast<float *>(ws + w.stats);
     p.stats = L.norm ? reinterpret_cast<float *>(ws + w.part_lse) : stats;
     p.status = reinterpret_cast<int *>(ws + w.status);
-    p.queue = reinterpret_cast<int *>(ws + w.status + 128);
+    p.queue = queue_slot(ws, 0);
     SPAVA_TRY(L.d == 128 ? launch_attn<128, true>(p, st) : launch_attn<64, true>(p, st));
     if (!L.norm) return SPAVA_OK;
     const int rows = L.Hq * L.q;
@@ -476,7 +482,7 @@ spava_status run_merge(const Layer &L, void *o, float *lse, char *ws, cudaStream
 spava_status run_attn(const Layer &L, const void *q, const void *k, const void *v, const void *pk,
                       const void *pv, void *o, float *lse, char *ws, cudaStream_t st,
                       int row_lo = 0, int row_hi = INT32_MAX, unsigned kinds = kAllKinds,
-                      bool merge = true) {
+                      bool merge = true, int slot = 0) {
     const WsLayout w = ws_layout(L);
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
@@ -493,7 +499,7 @@ spava_status run_attn(const Layer &L, const void *q, const void *k, const void *
     p.part_O = reinterpret_cast<float *>(ws + w.part_o);
     p.part_lse = reinterpret_cast<float *>(ws + w.part_lse);
     p.status = reinterpret_cast<int *>(ws + w.status);
-    p.queue = reinterpret_cast<int *>(ws + w.status + 128);  // inside the 256-byte status block
+    p.queue = queue_slot(ws, slot);
     SPAVA_TRY(L.d == 128 ? launch_attn<128, false>(p, st) : launch_attn<64, false>(p, st));
     if (!merge || L.N - L.q < row_lo || L.N > row_hi) return SPAVA_OK;  // query block not in this range
     return run_merge(L, o, lse, ws, st);
@@ -744,6 +750,23 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
         return e;
     };
     const bool chunkwise = L.norm == 0;
+    // The chunk pipeline's own streams: scoring (at the device's highest
+    // priority, so that its CTAs take the first SMs an attention launch frees)
+    // and two for the attention launches.  Destroying a stream with work still
+    // queued is safe: it is released once that work completes.
+    cudaStream_t side[3] = {nullptr, nullptr, nullptr};
+    if (chunkwise) {
+        int prio_least = 0, prio_greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&prio_least, &prio_greatest) != cudaSuccess)
+            return cuda_fail(cudaGetLastError());
+        for (int i = 0; i < 3; ++i)
+            if (cudaStreamCreateWithPriority(&side[i], cudaStreamNonBlocking,
+                                             i == 0 ? prio_greatest : prio_least) != cudaSuccess) {
+                const cudaError_t e = cudaGetLastError();
+                for (int j = 0; j < i; ++j) cudaStreamDestroy(side[j]);
+                return cuda_fail(e);
+            }
+    }
     auto body = [&]() -> spava_status {
         cudaEvent_t e_start = new_event();
         if (rc != SPAVA_OK) return rc;
@@ -782,58 +805,75 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
             // the PV product, and 0 x (a NaN or Inf not yet overwritten) is NaN.
             // So a region's attention waits until every row its tiles touch has
             // arrived.
-            auto wait_rows = [&](int end) -> spava_status {  // rows [0, end) on the device
-                if (end > L.off[L.n_chunks]) return cuda_ok(cudaStreamWaitEvent(st, e_query, 0));
+            auto wait_rows = [&](cudaStream_t s, int end) -> spava_status {  // rows [0, end) on the device
+                if (end > L.off[L.n_chunks]) return cuda_ok(cudaStreamWaitEvent(s, e_query, 0));
                 int c = 0;
                 while (L.off[c + 1] < end) ++c;
-                return cuda_ok(cudaStreamWaitEvent(st, e_chunk[c], 0));
+                return cuda_ok(cudaStreamWaitEvent(s, e_chunk[c], 0));
             };
             auto tiles_end = [&](int r0, int r1) { return std::min(L.N, r0 + kRowTile * cdiv(r1 - r0, kRowTile)); };
             const bool select = L.n_chunks > 1 && L.l > 0;
             float *scores = reinterpret_cast<float *>(w + lay.scores);
             const float *stats = reinterpret_cast<const float *>(w + lay.stats);
             int32_t *idx = reinterpret_cast<int32_t *>(w + lay.idx);
+            // Scoring runs on its own stream, ahead of the attention; the
+            // attention launches alternate between two streams, each waiting only
+            // for its rows and the passing blocks before them, so that a launch's
+            // persistent CTAs take over the SMs its predecessor's tail frees.
+            cudaStream_t ss = side[0];
+            for (int i = 0; i < 3; ++i) SPAVA_CUDA(cudaStreamWaitEvent(side[i], e_start, 0));
             // The packed passing blocks fill up chunk by chunk, and a packed
             // segment's last tile reads past its end into blocks not yet written:
             // those rows start as zeros, not as whatever the workspace held.
             if (select) {
                 const size_t packed = 2 * size_t(L.Hkv) * L.L * L.d;
-                SPAVA_CUDA(cudaMemsetAsync(w + lay.pk, 0, packed, st));
-                SPAVA_CUDA(cudaMemsetAsync(w + lay.pv, 0, packed, st));
+                SPAVA_CUDA(cudaMemsetAsync(w + lay.pk, 0, packed, ss));
+                SPAVA_CUDA(cudaMemsetAsync(w + lay.pv, 0, packed, ss));
             }
-            SPAVA_CUDA(cudaStreamWaitEvent(st, e_anchor, 0));
-            if (!select) SPAVA_TRY(run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, st));  // anchor rows
-            auto attend = [&](int r0, int r1) -> spava_status {
+            SPAVA_CUDA(cudaStreamWaitEvent(ss, e_anchor, 0));
+            if (!select) SPAVA_TRY(run_pack(L, k, v, idx, w + lay.pk, w + lay.pv, ss));  // anchor rows
+            cudaEvent_t e_init = new_event();
+            if (rc != SPAVA_OK) return rc;
+            SPAVA_CUDA(cudaEventRecord(e_init, ss));
+            int turn = 0;
+            auto attend = [&](int r0, int r1, cudaEvent_t after) -> spava_status {
                 if (r1 <= r0) return SPAVA_OK;
-                SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, want_lse ? lse : nullptr, w, st,
-                                   r0, r1));
+                cudaStream_t sa = side[1 + turn];
+                const int slot = 1 + turn;
+                turn ^= 1;
+                SPAVA_TRY(wait_rows(sa, tiles_end(r0, r1)));
+                SPAVA_CUDA(cudaStreamWaitEvent(sa, after, 0));
+                SPAVA_TRY(run_attn(L, q, k, v, w + lay.pk, w + lay.pv, o, want_lse ? lse : nullptr, w, sa,
+                                   r0, r1, kAllKinds, true, slot));
                 cudaEvent_t e = new_event();
                 if (rc != SPAVA_OK) return rc;
-                SPAVA_CUDA(cudaEventRecord(e, st));
+                SPAVA_CUDA(cudaEventRecord(e, sa));
                 rows.emplace_back(r0, r1);
                 computed.push_back(e);
                 return SPAVA_OK;
             };
-            if (L.a > 0) {
-                SPAVA_TRY(wait_rows(tiles_end(0, L.a)));
-                SPAVA_TRY(attend(0, L.a));
-            }
+            if (L.a > 0) SPAVA_TRY(attend(0, L.a, e_init));
+            cudaEvent_t sel_before = e_init;  // the passing blocks of every chunk before c
             for (int c = 0; c < L.n_chunks; ++c) {
-                SPAVA_CUDA(cudaStreamWaitEvent(st, e_chunk[c], 0));
+                cudaEvent_t sel_c = sel_before;
                 if (select && c < L.n_chunks - 1) {
                     // this chunk's passing block: the same kernels as the whole
                     // layer's front, restricted to chunk c
                     Layer Lc = L;
                     Lc.own = 1ULL << c;
-                    SPAVA_TRY(run_stats(Lc, q, k, w, st));
-                    SPAVA_TRY(run_scores_ws(Lc, q, k, stats, scores, w, st, true, idx, v, w + lay.pk,
+                    SPAVA_CUDA(cudaStreamWaitEvent(ss, e_chunk[c], 0));
+                    SPAVA_TRY(run_stats(Lc, q, k, w, ss));
+                    SPAVA_TRY(run_scores_ws(Lc, q, k, stats, scores, w, ss, true, idx, v, w + lay.pk,
                                             w + lay.pv, c == 0));
+                    sel_c = new_event();
+                    if (rc != SPAVA_OK) return rc;
+                    SPAVA_CUDA(cudaEventRecord(sel_c, ss));
                 }
-                SPAVA_TRY(wait_rows(tiles_end(L.off[c], L.off[c + 1])));
-                SPAVA_TRY(attend(L.off[c], L.off[c + 1]));
+                // chunk 0's scoring launch also copies the anchor rows
+                SPAVA_TRY(attend(L.off[c], L.off[c + 1], c == 0 ? sel_c : sel_before));
+                sel_before = sel_c;
             }
-            SPAVA_CUDA(cudaStreamWaitEvent(st, e_query, 0));
-            SPAVA_TRY(attend(q0, L.N));
+            SPAVA_TRY(attend(q0, L.N, sel_before));
         } else {
             // Row-normalised scores need every segment's statistics first: K and
             // the query block's Q rows go up first, then V, then the Q rows of
@@ -884,6 +924,8 @@ spava_status spava_prefill_attention_host(const spava_config *cfg, const void *q
     // Destroying a recorded event is safe: its resources go once it completes.
     for (auto e : ev)
         if (e) cudaEventDestroy(e);
+    for (auto s : side)
+        if (s) cudaStreamDestroy(s);
     return rc;
 }
 
