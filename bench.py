@@ -41,6 +41,9 @@ sys.path.insert(0, ROOT)
 from sequence_sparse_attention_b200.synth import WORKLOADS, chunk_offsets, make_inputs  # noqa: E402
 
 METRIC = "approx-attn prefill tokens/s per layer on 1 B200; % BF16 tensor peak"
+# The spec sheet's dense bf16 tensor figure for one B200 (its 2:4-sparse
+# figure halved): context beside the measured peaks.
+NOMINAL_BF16_DENSE_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # Kernels one spava_prefill_attention call launches: the anchor rows and
 # query partials (attention kernel), scoring fused with top-l and gather, the
@@ -379,6 +382,7 @@ def run_ours(args, world, rank, local):
                 "kernel": "attn_kernel<128> + query merge (spava_attn)",
                 "peak_kind": f"{pe} bf16 dense GEMM, burst",
                 "frac_of_sustained_peak": achieved / sustained,
+                "frac_of_nominal_dense_peak": achieved / NOMINAL_BF16_DENSE_TFLOPS,
                 "tflops_per_ghz": achieved / (sm_mhz / 1e3) if sm_mhz else None,
                 "frac_of_tensor_pipe_at_sampled_clock": achieved / pipe_at_clock if pipe_at_clock else None,
                 "launch_ms": per["attn"],
@@ -403,6 +407,17 @@ def run_ours(args, world, rank, local):
                  for k, b in sel_bytes.items()}
     phase_bytes = sum(sel_bytes.values())
     phase_ms = per["score"] + per["topk"] + per["pack"]
+    # Scoring is a contraction with one exponential per (query row, head, key),
+    # done twice (the statistics pass, then the scores): its TFLOP/s and
+    # exponentials per second, the latter against the MUFU rate at the sampled
+    # clock (16 per SM per clock; a quarter of the scoring pass's exponentials
+    # run on the FMA pipe instead, so the fraction can pass 1).
+    triples = w.Hq * w.q * scored
+    score_s = per["score"] / 1e3
+    selection["score"]["TFLOP/s"] = 2 * 2 * w.d * triples / score_s / 1e12
+    selection["score"]["exp/s"] = 2 * triples / score_s
+    selection["score"]["frac_of_mufu_at_sampled_clock"] = (
+        2 * triples / score_s / (n_sm * 16 * sm_mhz * 1e6) if sm_mhz else None)
     selection["phase"] = {"bytes": phase_bytes, "ms": phase_ms,
                           "GB/s": phase_bytes / (phase_ms / 1e3) / 1e9,
                           "frac_of_hbm": phase_bytes / (phase_ms / 1e3) / 1e9 / hbm}
