@@ -102,6 +102,23 @@ def test_pointer_and_workspace_checks_before_launch():
     assert status("spava_attn", lay, fake, fake, fake, fake, fake, fake, None, base + 16, ws_bytes, None) == 3
     assert status("spava_prefill_attention", lay, fake, fake, None, fake, None, None, base, ws_bytes, None) == 1
     assert status("spava_score", lay, fake, fake, fake, base, 16, None) == 4
+    # selection and gather: missing scores, misaligned indices, misaligned packed rows
+    assert status("spava_topk_select", lay, None, fake, None) == 1
+    assert status("spava_topk_select", lay, fake, fake + 4, None) == 3
+    assert status("spava_pack_passing", lay, fake, fake, fake, fake + 8, fake, None) == 3
+    assert status("spava_pack_passing", lay, fake, None, fake, fake, fake, None) == 1
+    # host-buffer entry point: host and device pointers, then the workspace, all
+    # checked before the first copy or stream is made
+    host = fake  # any non-null host address; never read on these paths
+    args = [host, host, host, host, None, fake, fake, fake, fake, None, base, ws_bytes, None, None]
+    bad = list(args); bad[1] = None                      # k_host missing
+    assert status("spava_prefill_attention_host", lay, *bad) == 1
+    bad = list(args); bad[5] = fake + 2                  # q misaligned
+    assert status("spava_prefill_attention_host", lay, *bad) == 3
+    bad = list(args); bad[11] = ws_bytes - 1             # workspace short
+    assert status("spava_prefill_attention_host", lay, *bad) == 4
+    bad = list(args); bad[10] = None                     # workspace missing
+    assert status("spava_prefill_attention_host", lay, *bad) == 4
 
 
 def test_workspace_and_packed_sizes():
