@@ -275,3 +275,30 @@ def test_host_buffers_back_to_back():
     for (Q, K, V, _), (_, _, _, oh) in zip(ins, hosts):
         O_dev, _, _ = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda())
         assert torch.equal(oh.view(torch.int16), O_dev.cpu().view(torch.int16))
+
+
+def test_host_buffers_on_a_caller_stream():
+    """The caller computes on its own (non-default) stream: the pipelined host
+    call ends on that stream, so synchronising it alone is enough to read the
+    host outputs, which equal the device entry point's bytes."""
+    w = CASES["g7"]
+    Q, K, V, _ = make_inputs(w)
+    sp = Spava(Layout.from_workload(w))
+    qh, kh, vh = Q.pin_memory(), K.pin_memory(), V.pin_memory()
+    oh = torch.full_like(Q, 7.0).pin_memory()
+    lh = torch.full((w.Hq, w.N), 7.0, dtype=torch.float32).pin_memory()
+    qd, kd, vd = (torch.full_like(x, float("nan"), device="cuda") for x in (Q, K, V))
+    od = torch.full_like(qd, float("nan"))
+    ld = torch.empty((w.Hq, w.N), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    compute, copies = torch.cuda.Stream(), torch.cuda.Stream()
+    with torch.cuda.stream(compute):
+        for _ in range(2):
+            sp.prefill_attention_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, copy_stream=copies)
+    compute.synchronize()
+    oh_c, lh_c = oh.clone(), lh.clone()
+    torch.cuda.synchronize()
+    device_clean(sp)
+    O_dev, lse_dev, _ = sp.prefill_attention(Q.cuda(), K.cuda(), V.cuda())
+    assert torch.equal(oh_c.view(torch.int16), O_dev.cpu().view(torch.int16))
+    assert torch.equal(lh_c, lse_dev.cpu())
