@@ -20,7 +20,11 @@
 //   warp  9    MMA issuer (warps 10-11 only complete its warpgroup), per key tile j:
 //                PV_A(j)  S_A(j+1)  PV_B(j)  S_B(j+1)
 //              so S_X(j+1) enters the tensor pipe right behind PV_X(j) while the
-//              other tile's softmax is running.
+//              other tile's softmax is running.  The whole warp runs the loop
+//              (lane 0 issues): it meets tile X's softmax warps at the named
+//              barrier that announces P_X(j).
+// Hand-offs: TMA and MMA completions reach the other roles through mbarriers
+// (bounded waits); P_X(j) reaches the MMA warp through a named barrier.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
 // P_X(j) (bf16 pairs) goes to S_X's columns [0,64) once the softmax holds all of
 // S_X(j) in registers.  The tcgen05.mma operations of one thread run in issue
@@ -75,7 +79,7 @@ struct AttnSmem {
     static constexpr int kOffK = 2 * kTile;
     static constexpr int kOffV = kOffK + KS * kTile;
     static constexpr int kOffBar = kOffV + VS * kTile;
-    static constexpr int kNumBar = 1 + 2 * KS + 2 * VS + 6 + 1;
+    static constexpr int kNumBar = 1 + 2 * KS + 2 * VS + 4 + 1;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
     static constexpr int kBytes = kOffMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -98,6 +102,17 @@ static_assert(128 * kRegsIo + 256 * kRegsSoftmax <= kAttnThreads * kLaunchRegs,
               "register split above the CTA's pool");
 constexpr int kColO = 256;  // O_A; O_B at kColO + 128
 constexpr int kItemBar = 1;  // named barrier of all threads between work items
+// P_X(j) is in TMEM (or, in the statistics pass, S_X(j) has been read): named
+// barrier kPBar + X between tile X's four softmax warps (bar.arrive) and the
+// whole MMA warp (bar.sync).  A hardware barrier hands off in ~130 cycles, an
+// mbarrier's arrive-to-wake in ~350.  It has no timeout, so arrivals and syncs
+// pair one for one by construction: the MMA warp syncs P_X(j) only after it has
+// issued S_X(j), and the softmax warps arrive for step j only after S_X(j) has
+// completed, waiting for it without regard to other roles' aborts (their own
+// bounded wait gives up only if a committed MMA never completes).  At most one
+// arrival is ever pending, since the next S needs the sync first.
+constexpr int kPBar = 2;
+constexpr int kPBarThreads = 4 * 32 + 32;
 
 // Work items of a region (one group): row tiles 2p and 2p+1 of one query head;
 // when the region has an odd number of row tiles, its last tile (the costliest,
@@ -214,8 +229,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     uint64_t *v_full = k_empty + KS;
     uint64_t *v_empty = v_full + VS;
     uint64_t *s_full = v_empty + VS;  // [2]: S_X(j) in TMEM
-    uint64_t *p_full = s_full + 2;    // [2]: P_X(j) in TMEM
-    uint64_t *o_done = p_full + 2;    // [2]: the last PV_X has completed
+    uint64_t *o_done = s_full + 2;    // [2]: the last PV_X has completed
     uint64_t *mma_drain = o_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SM::kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + SM::kOffMisc + 4);
@@ -242,7 +256,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         }
         for (int i = 0; i < 2; ++i) {
             init(&s_full[i], 1);
-            init(&p_full[i], 128);
             init(&o_done[i], 1);
         }
         init(mma_drain, 1);
@@ -363,7 +376,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the loop (it takes part in the P barriers, which
+        // count whole warps); lane 0 alone issues the tcgen05 operations, and
+        // every lane's wait result is combined so that the warp stays converged.
+        {
+            const bool leader = lane == 0;
+            auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, ab));
+            };
+            auto commit = [&](uint64_t *bar) {
+                if (leader) tc_commit(bar);
+            };
             // Descriptors built once; a K-step or a ring stage adds its byte
             // offset / 16 to the start-address field.
             constexpr int NK = D / 16;
@@ -379,6 +402,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
             }
             // S_X(j) = Q_X K_j^T into TMEM columns [128x, 128x+128).
             auto mma_s = [&](int x, int j) {
+                if (!leader) return;
                 const uint64_t kd = k_desc + static_cast<uint64_t>(((j % KS) * SM::kTile) >> 4);
                 const uint32_t d_s = tmem + x * kKeyTile;
 #pragma unroll
@@ -392,6 +416,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
             // O_X += P_X(j) V_j.  K-step kb covers keys 16kb..16kb+15: P columns
             // +8kb inside S_X, V rows +2048 B.
             auto mma_pv = [&](int x, int j) {
+                if (!leader) return;
                 const uint32_t a_p = tmem + x * kKeyTile;
                 const uint64_t vd = v_desc + static_cast<uint64_t>(((j % VS) * SM::kTile) >> 4);
                 const uint32_t d_o = tmem + kColO + x * 128;
@@ -400,12 +425,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 mma_ts_x4(d_o, a_p + 32, a_p + 40, a_p + 48, a_p + 56, vd + 512, vd + 640, vd + 768,
                           vd + 896, kIdescPV, 1u);
             };
-            bool ok = mbar_wait(q_full, 0, ab) && (T == 0 || mbar_wait(&k_full[0], 0, ab));
+            bool ok = wait(q_full, 0) && (T == 0 || wait(&k_full[0], 0));
             tc_fence_after();
             if (ok && T > 0) {
                 if (TA > 0) mma_s(0, 0);
                 if (TB > 0) mma_s(1, 0);
-                tc_commit(&k_empty[0]);
+                commit(&k_empty[0]);
             }
             // Statistics only: S_X(j+1) as soon as the softmax has read S_X(j).
             for (int j = 0; STATS && ok && j < T; ++j) {
@@ -415,12 +440,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                 for (int x = 0; x < 2; ++x) {
                     const int TX = x ? TB : TA;
                     if (ok && j < TX) {
-                        ok = mbar_wait(&p_full[x], j & 1, ab);
-                        if (!ok) break;
+                        __syncwarp();
+                        bar_sync(kPBar + x, kPBarThreads);
                         tc_fence_after();
                         if (kn < TX) {
                             if (!k_seen) {
-                                ok = mbar_wait(&k_full[ks], (kn / KS) & 1, ab);
+                                ok = wait(&k_full[ks], (kn / KS) & 1);
                                 if (!ok) break;
                                 tc_fence_after();
                                 k_seen = true;
@@ -430,24 +455,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                     }
                 }
                 if (!ok) break;
-                if (k_seen) tc_commit(&k_empty[ks]);
+                if (k_seen) commit(&k_empty[ks]);
             }
             for (int j = 0; !STATS && ok && j < T; ++j) {
                 const int vs = j % VS, kn = j + 1, ks = kn % KS;
-                if (!mbar_wait(&v_full[vs], (j / VS) & 1, ab)) break;
+                if (!wait(&v_full[vs], (j / VS) & 1)) break;
                 bool k_seen = false;
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     const int TX = x ? TB : TA;
                     if (ok && j < TX) {
-                        ok = mbar_wait(&p_full[x], j & 1, ab);
-                        if (!ok) break;
+                        __syncwarp();
+                        bar_sync(kPBar + x, kPBarThreads);
                         tc_fence_after();
                         mma_pv(x, j);
-                        if (j + 1 == TX) tc_commit(&o_done[x]);
+                        if (j + 1 == TX) commit(&o_done[x]);
                         if (kn < TX) {
                             if (!k_seen) {
-                                ok = mbar_wait(&k_full[ks], (kn / KS) & 1, ab);
+                                ok = wait(&k_full[ks], (kn / KS) & 1);
                                 if (!ok) break;
                                 tc_fence_after();
                                 k_seen = true;
@@ -457,11 +482,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                     }
                 }
                 if (!ok) break;
-                tc_commit(&v_empty[vs]);
-                if (k_seen) tc_commit(&k_empty[ks]);
+                commit(&v_empty[vs]);
+                if (k_seen) commit(&k_empty[ks]);
             }
             // No MMA may still be running when TMEM is released.
-            tc_commit(mma_drain);
+            commit(mma_drain);
             mbar_wait_drain(mma_drain, 0);
         }
         __syncwarp();
@@ -500,7 +525,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
             const int lim = lim_end - key0;  // keys [0, lim) of this tile are valid for row r
             cur.advance(segs);
 
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], j & 1, ab));
+            // Not cut short by another role's abort: once the MMA warp has issued
+            // S_X(j) it will wait on this tile's P barrier, and only a completed
+            // S_X(j) may be answered there (or the barrier would be left short).
+            ok = __all_sync(0xffffffffu, mbar_wait_own(&s_full[x], j & 1, ab));
             if (!ok) break;
             tc_fence_after();
             float xs[kKeyTile];
@@ -518,7 +546,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
             }
             if (STATS) {  // S_X(j) is in registers: the next S may overwrite it
                 tc_fence_before();
-                mbar_arrive(&p_full[x]);
+                bar_arrive(kPBar + x, kPBarThreads);
             }
             if (lim < kKeyTile) {  // only tiles crossing a segment end or the diagonal
 #pragma unroll
@@ -572,7 +600,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
             if (!STATS) {
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&p_full[x]);
+                bar_arrive(kPBar + x, kPBarThreads);
             }
             const float2 pss = fadd2(ps[0], ps[1]);
             l_run = __fadd_rn(l_run, __fadd_rn(pss.x, pss.y));

@@ -77,6 +77,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     }
 }
 
+// Bounded wait that ignores the CTA's abort flag: it returns false only after
+// its own time limit (then flags the CTA and the workspace).
+__device__ __forceinline__ bool mbar_wait_own(uint64_t *bar, uint32_t parity, const AbortState &ab) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            *ab.cta_flag = 1;
+            atomicOr(ab.status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
 // Drain wait used on the abort path: bounded, never flags.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     const long long t0 = clock64();
@@ -249,6 +266,10 @@ __device__ __forceinline__ void reg_dealloc() {
 // ------------------------------------------------------------------ named barriers
 __device__ __forceinline__ void bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Arrive on named barrier `id` (n threads in all) without waiting.
+__device__ __forceinline__ void bar_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 // ------------------------------------------------------------------ math
 // Hardware base-2 exponential (MUFU.EX2), flush-to-zero approximate.
