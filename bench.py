@@ -55,8 +55,8 @@ KERNELS_PER_SPLIT_STEP = 6
 # DRAM traffic of one attention launch on the 128K layer (dram__bytes_read.sum
 # + dram__bytes_write.sum of a single-pass ncu capture); valid only while the
 # sources that decide it hash to the value it was taken with (KERNEL_FILES).
-PROFILED_TRAFFIC = {"kernel_sha256": "7a2e744835e1d69e8dfcf3f1a7fa59425e340bc982e4f26ca0046c4e62311cc6",
-                    "bytes_per_launch": 3277795584 + 1261207296, "workload": "128k"}
+PROFILED_TRAFFIC = {"kernel_sha256": "d74482952a1f6e0b8adfcf54662d3e6c85f4b0e170f3983994054cd57cafad9f",
+                    "bytes_per_launch": 3090140672 + 1257348096, "workload": "128k"}
 KERNEL_FILES = ("attn_kernel.cuh", "plan.cuh", "sm100.cuh")  # what decides the attention launch
 
 
